@@ -1,0 +1,387 @@
+#!/usr/bin/env python3
+"""Benchmark of the decode-attention stack (q_rotate, kv_append,
+paged_decode_attn, attn_combine for every full-attention layer) on one B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...        # the oracle on the host cores
+
+A step is one decode step of the whole attention stack: for each of the 16
+layers, rotate the query (q4_0), append this step's K/V token, run the split-K
+decode over the full context and combine the splits.  Inputs are resident in
+HBM when the timed region starts; the KV pool (4.83 GB for the default
+workload) is larger than L2, so no flush is needed between steps.  Under
+torchrun each rank runs an independent replica (weak scaling, no collective
+on the data path); the reported time is the max over ranks.
+
+One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV GB/s & % HBM peak; attn-stack tokens/s at 262K ctx (1 B200)"
+DEFAULT_WORKLOAD = "qwen27b_q4_0_262k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("kvq_decode.cu", "kvq_internal.cuh"):
+        h.update(open(os.path.join(ROOT, "quantized_kv_cache_17_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_tag: str, workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(f"{kernel_tag}:{workload}")
+        if e and e.get("source_hash") == decode_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU during the timed region."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9 or (self.uuid and self.uuid not in parts[0]):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def cpu_oracle_rate(fmt: str, G: int, codes_list, qp_list, budget_s: float):
+    """Time the oracle (single thread, as it stands) on the given (layer, KV
+    head) groups; returns (KV GB/s, token-kvheads/s, seconds, groups done)."""
+    import oracle
+    t0 = time.perf_counter()
+    done_bytes = 0
+    done_tok = 0
+    n = 0
+    per_tok = oracle.format_bytes_per_token_head(fmt)
+    for codes, qp in zip(codes_list, qp_list):
+        kc, ks, vc, vs = codes
+        oracle.attn_decode(fmt, qp, kc, ks, vc, vs)
+        done_tok += kc.shape[0]
+        done_bytes += kc.shape[0] * per_tok
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done_bytes / dt / 1e9, done_tok / dt, dt, n
+
+
+def run_reference(args):
+    """The oracle on the host cores, each step a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import kvq_inputs
+    import oracle
+    w = kvq_inputs.workload(args.workload)
+    layer, b, g = 0, 0, 0
+    T_sample = min(w.seq_lens[-1], 8192)
+    k = w.k_rows(layer, b, 0, T_sample)[:, g]
+    v = w.v_rows(layer, b, 0, T_sample)[:, g]
+    codes = oracle.append_rows(w.fmt, k, v)
+    qp = oracle.q_prepare(w.fmt, w.q_row(layer, b)[g * w.group:(g + 1) * w.group])
+    per_tok = oracle.format_bytes_per_token_head(w.fmt)
+    for _ in range(args.warmup):
+        oracle.attn_decode(w.fmt, qp, *codes)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.attn_decode(w.fmt, qp, *codes)
+        times.append(time.perf_counter() - t0)
+    dt = sum(times) / len(times)
+    gbs = T_sample * per_tok / dt / 1e9
+    sample = (f"oracle fp64 attention of one (layer, KV head) group ({w.group} query heads) over "
+              f"{T_sample} tokens of {w.name}, codes from the oracle's own append; single thread")
+    line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "format": w.fmt, "seq_lens": w.seq_lens, "layers": w.n_layers,
+                       "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 256},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import kvq_inputs
+    import quantized_kv_cache_17_b200 as kvq
+    from kvq_inputs import device as kdev
+
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+
+    kvq.lib()   # fails loudly if the library is missing
+    w = kvq_inputs.workload(args.workload)
+    if args.layers:
+        w = kvq_inputs.scaled(w, w.seq_lens, n_layers=args.layers, name=w.name)
+    L = w.n_layers
+    fmt = w.fmt
+    dw = kdev.build_pool(w, extra_slots=0)
+    q, k_new, v_new, pos = kdev.step_inputs(w, list(range(L)))
+    plan, info = kvq.decode_plan(dw.pool.desc, w.seq_lens, dw.page_table.shape[1], args.n_ctas)
+    plan_d = torch.from_numpy(plan).cuda()
+    ws = torch.empty(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    q_rot = torch.empty_like(q)
+    out_bf = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+    out_f = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    rot_q, rot_v = kvq.rotated_q(fmt), kvq.rotated_v(fmt)
+    use_alu = args.decode == "alu"
+    layout = kvq.pool_layout(dw.pool.desc)
+    kv_bytes_layer = sum(w.seq_lens) * w.n_kv_heads * layout.bytes_per_token_head
+
+    def layer_step(l, dec_events=None):
+        qq = q[l]
+        if rot_q:
+            kvq.q_rotate(qq, q_rot[l], stream)
+            qq = q_rot[l]
+        kvq.kv_append(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, status=status, stream=stream)
+        if dec_events is not None:
+            dec_events[0].record(stream)
+        kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, stream, cudacore=use_alu)
+        if dec_events is not None:
+            dec_events[1].record(stream)
+        kvq.attn_combine(ws, plan_d, info, rot_v, out_bf[l], out_f[l], stream)
+
+    def step(evs=None):
+        for l in range(L):
+            layer_step(l, evs[l] if evs is not None else None)
+
+    launches_per_layer = 3 + (1 if rot_q else 0)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"kernel status {status.item()}"
+
+    uuid = ""
+    try:
+        uuid = str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    dec_evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+               for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    torch.cuda.cudart().cudaProfilerStart()      # an ncu launch list with --profile-from-start off sees only this region
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(dec_evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    torch.cuda.cudart().cudaProfilerStop()
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = [e[0].elapsed_time(e[1]) for st in dec_evs for e in st]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+
+    # ---- end to end: host buffers, copies inside the timed region ---------------
+    q_h = q.cpu().pin_memory()
+    k_h = k_new.cpu().pin_memory()
+    v_h = v_new.cpu().pin_memory()
+    o_h = torch.empty(out_bf.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = q_h.numel() * 4 + k_h.numel() * 4 + v_h.numel() * 4
+    d2h = o_h.numel() * 2
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for s in range(args.steps):
+        q.copy_(q_h, non_blocking=True)
+        k_new.copy_(k_h, non_blocking=True)
+        v_new.copy_(v_h, non_blocking=True)
+        step()
+        o_h.copy_(out_bf, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+    assert int(status.item()) == 0, f"kernel status {status.item()}"
+
+    if dist is not None:
+        t = torch.tensor([elapsed_ms, e2e_ms, dec_avg_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms, dec_avg_ms = t.tolist()
+
+    ms_per_step = elapsed_ms / args.steps
+    kv_bytes_step = kv_bytes_layer * L
+    value = world * kv_bytes_step / (ms_per_step * 1e-3) / 1e9
+    e2e_value = world * kv_bytes_step / (e2e_ms / args.steps * 1e-3) / 1e9
+    tok_s = world * w.batch / (ms_per_step * 1e-3)
+    peak, peak_kind = peaks()
+    achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
+    kernel_tag = "decode_alu" if use_alu else "decode_mma"
+    traffic = ncu_traffic(kernel_tag, w.name)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        from tests import kvq_layout
+        codes_list, qp_list = [], []
+        for g in range(min(args.cpu_groups, w.n_kv_heads)):
+            b = len(w.seq_lens) - 1
+            codes_list.append(kvq_layout.gather_sequence(fmt, dw.pool.buf, layout, L - 1, g, dw.page_table_host[b],
+                                                         w.seq_lens[b]))
+            qp_list.append(oracle.q_prepare(fmt, q[L - 1, b, g * w.group:(g + 1) * w.group].cpu().numpy()))
+        gbs, tok_rate, dt, n = cpu_oracle_rate(fmt, w.group, codes_list, qp_list, args.cpu_budget)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"oracle fp64 attention of {n} (layer, KV head) groups ({w.group} query heads each) over "
+                         f"{w.seq_lens[-1]} tokens of {w.name}, codes read back from the GPU pool; "
+                         f"single thread, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32 (codes u4/i8, fp16 scales, fp16 tensor-core "
+                "operands with hi/lo split)" if not use_alu else "f32",
+                "data": "synthetic (seeded counter-based generator; shapes and value distributions of the pages' "
+                        "workloads)",
+                "config": {"workload": w.name, "format": fmt, "seq_lens": w.seq_lens, "layers": L,
+                           "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 256, "page_tokens": 256,
+                           "decode_kernel": kernel_tag, "n_units": info.n_units, "chunk_tokens": info.chunk_tokens,
+                           "kv_bytes_per_step": kv_bytes_step,
+                           "l2": "no flush: the 16-layer KV pool read per step is larger than L2",
+                           "parallelism": f"replicas x{world}"},
+                "attn_stack_tok_s": round(tok_s, 2),
+                "us_per_layer_step": round(ms_per_step * 1e3 / L, 3),
+                "us_decode_per_layer": round(dec_avg_ms * 1e3, 3),
+                "pct_of_8tbs_spec": round(100 * value / world / 8000.0, 2),
+                "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                             "frac": round(achieved / peak, 4), "traffic": traffic,
+                             "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                             if peak_kind == "measured" else "fallback 6.65 TB/s",
+                             "bytes_per_launch": kv_bytes_layer,
+                             "kernel": kernel_tag},
+                "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
+                "gpu_launches": args.steps * L * launches_per_layer,
+                "clocks": clocks,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--decode", default="mma", choices=["mma", "alu"])
+    ap.add_argument("--n-ctas", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-groups", type=int, default=4)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * kvq.h - C ABI of the quantized paged decode-attention library (B200, sm_100a).
+ *
+ * One decode step of a full-attention GQA layer over a long KV cache held in
+ * 4-bit or 8-bit form:
+ *
+ *   q_rotate                      rotate the query by the same transform as K
+ *   kv_append                     rotate, quantise and scatter the step's new K/V
+ *   paged_decode_attn_{int8,q4_0,k8v4}
+ *                                 split-K attention over the page table
+ *   attn_combine                  merge the splits, un-rotate, write bf16 + f32
+ *
+ * Sources (web pages, cited by title and section):
+ *  [Strata] "KV 沉进内存、显存减半：Strata 让 12 GB 显卡跑满 262K 上下文"
+ *           (hotelren.com news 6161890).  Section "4-bit KV 缓存：先旋转，再压到
+ *           4-bit": Q, K and V pass through a 256-point Walsh-Hadamard rotation
+ *           before 4-bit storage, scores are unchanged because <Hq,Hk> = <q,k>,
+ *           the output is mixed over rotated V and multiplied by H again.
+ *           Section "三种 KV 格式横向对比": formats int8 (default), q4_0 and k8v4
+ *           (K 8-bit, V rotated then 4-bit).  Section "KV 从显存搬进内存之后发生了
+ *           什么": KV in fixed pages addressed through a residency table.
+ *  [Guide]  anozoder wiki "qwen38-27b-quant-vram-2026", section "一": the 27B
+ *           full-attention shape (24 Q heads, 4 KV heads, head_dim 256, 16
+ *           layers) and the KV-size formula; section "二": the q4_0 block size.
+ *
+ * Conventions (all entry points):
+ *  - Every function returns KVQ_OK (0) or a negative KVQ_E* code and never
+ *    throws.  Argument errors are detected on the host before any launch.
+ *  - The caller owns every buffer.  The library never allocates device or host
+ *    memory.  Device pointers must be 16-byte aligned (KVQ_EALIGN otherwise).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream); all device
+ *    work is enqueued asynchronously on it.  KVQ_ECUDA reports a launch error
+ *    (cudaGetLastError after the launch).
+ *  - `status` (nullable, device int32) receives OR-ed KVQ_STATUS_* bits from
+ *    kernels that detect bad data (a page-table entry outside the pool, a plan
+ *    entry out of range, an internal wait that gave up).  Affected tokens are
+ *    skipped; nothing faults.  The caller clears it.
+ *  - head_dim and page_tokens are both 256.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_OK 0
+#define KVQ_EINVAL (-1)        /* bad argument value (null, range, shape) */
+#define KVQ_EUNSUPPORTED (-2)  /* shape or format this build does not handle */
+#define KVQ_EALIGN (-3)        /* a device pointer is not 16-byte aligned */
+#define KVQ_ECUDA (-4)         /* a CUDA runtime call or launch failed */
+#define KVQ_ESIZE (-5)         /* a caller buffer is smaller than required */
+
+#define KVQ_STATUS_BAD_SLOT 1u   /* page-table entry outside [0, n_pages) */
+#define KVQ_STATUS_BAD_PLAN 2u   /* plan entry inconsistent with the pool */
+#define KVQ_STATUS_TIMEOUT 4u    /* a pipeline wait exceeded its time limit */
+
+#define KVQ_HEAD_DIM 256
+#define KVQ_PAGE_TOKENS 256
+#define KVQ_MAX_GROUP 8          /* query heads per KV head handled by one CTA */
+
+/* KV formats ([Strata] "三种 KV 格式横向对比"):
+ *  KVQ_INT8  K and V int8, one fp16 scale per 64 values, no rotation.
+ *  KVQ_Q4_0  K and V rotated by H/16, then q4_0: one fp16 scale per 32 values,
+ *            codes 0..15 stored as nibbles ([Guide] "二" q4_0 block).
+ *  KVQ_K8V4  K int8 unrotated, V rotated then q4_0. */
+typedef enum { KVQ_INT8 = 0, KVQ_Q4_0 = 1, KVQ_K8V4 = 2 } kvq_format;
+
+typedef struct {
+    int32_t n_layers;     /* layers stored in the pool */
+    int32_t n_kv_heads;   /* KV heads per layer */
+    int32_t n_q_heads;    /* query heads per layer; a multiple of n_kv_heads */
+    int32_t head_dim;     /* must be 256 */
+    int32_t page_tokens;  /* must be 256 */
+    int32_t n_pages;      /* page slots per layer */
+    int32_t fmt;          /* kvq_format */
+} kvq_pool_desc;
+
+typedef struct {
+    void *base;           /* device memory of kvq_pool_bytes() bytes, caller-owned */
+    kvq_pool_desc desc;
+} kvq_pool;
+
+/* Byte layout of the pool.  The pool is [layer][slot][kv_head] page blocks;
+ * a page block is 32 tiles of 8 tokens; a tile holds, in this order, K codes,
+ * K scales, V codes and V scales of its 8 tokens (offsets below).  Inside a
+ * tile, codes and scales are arranged in the register-fragment order of the
+ * attention kernel; the exact element order is documented with the kernels and
+ * reproduced by the tests' layout decoder. */
+typedef struct {
+    int64_t tile_bytes;      /* bytes of one 8-token tile */
+    int64_t k_codes_off;     /* offsets of the four sections inside a tile */
+    int64_t k_scales_off;
+    int64_t v_codes_off;
+    int64_t v_scales_off;
+    int64_t page_bytes;      /* one (layer, slot, kv head) block = 32 tiles */
+    int64_t head_stride;     /* = page_bytes */
+    int64_t slot_stride;     /* = n_kv_heads * page_bytes */
+    int64_t layer_stride;    /* = n_pages * slot_stride */
+    int64_t total_bytes;     /* = n_layers * layer_stride */
+    int64_t bytes_per_token_head; /* algorithmic K+V bytes of one token of one KV head */
+} kvq_layout;
+
+/* Pool size and layout for a descriptor.  KVQ_EINVAL / KVQ_EUNSUPPORTED on a
+ * bad descriptor.  Host only; no CUDA call. */
+int kvq_pool_bytes(const kvq_pool_desc *desc, uint64_t *bytes);
+int kvq_pool_layout(const kvq_pool_desc *desc, kvq_layout *out);
+
+/* q_rotate: q_rot[i] = (H_256 / 16) q[i] for n_vec vectors of 256 fp32
+ * ([Strata] "4-bit KV 缓存": Q takes the same rotation as K so that
+ * <Hq, Hk> = <q, k>).  H is the Sylvester Hadamard matrix in natural order;
+ * the transform is eight butterfly stages h = 1, 2, ..., 128 mapping
+ * (x[i], x[i+h]) to (x[i] + x[i+h], x[i] - x[i+h]) in fp32 round-to-nearest
+ * without fused multiply-add, then an exact multiply by 1/16, so the result is
+ * bit-reproducible.  q and q_rot: device [n_vec][256] fp32, may alias.
+ * n_vec == 0 is a no-op. */
+int q_rotate(const float *q, float *q_rot, int64_t n_vec, void *stream);
+
+/* kv_append: encode n_rows new tokens into the pool of one layer.
+ *  k, v      device fp32 [n_rows][n_kv_heads][256]
+ *  row_seq   device int32 [n_rows] sequence of each row, or NULL (row i -> seq i)
+ *  row_pos   device int32 [n_rows] token position of each row in its sequence
+ *  page_table device int32 [n_seq][max_pages]: slot of page p of sequence s
+ * Per (row, kv head): rotate by H/16 where the format stores rotated data
+ * (q4_0: K and V; k8v4: V), quantise per block with the fp16 scale rounded to
+ * nearest and codes from round-half-even of a true division (q4_0: d =
+ * signed-max/-8, code = clamp(rint(x/d)+8, 0, 15); int8: d = max|x|/127, code =
+ * clamp(rint(x/d), -127, 127); a zero scale gives code 8 / 0), and store at
+ * slot page_table[seq][pos/256], token pos%256.  Codes and scales are
+ * bit-exact functions of the input.  A slot outside [0, n_pages) or a position
+ * outside [0, max_pages*256) sets KVQ_STATUS_BAD_SLOT and skips the row.
+ * Two rows writing the same (sequence, position) race. */
+int kv_append(const kvq_pool *pool, int layer, const float *k, const float *v, int64_t n_rows,
+              const int32_t *row_seq, const int32_t *row_pos, const int32_t *page_table,
+              int max_pages, int n_seq, int32_t *status, void *stream);
+
+/* Split plan for a batch of sequences (host only).  A plan partitions every
+ * (sequence, KV head) token range into work units of whole 64-token steps so
+ * that the number of units does not exceed n_ctas (0 = 2 per SM of the current
+ * device) and units are as even as possible; it also records, per
+ * (sequence, KV head), the first unit.  seq_len: host int32 [n_seq], the
+ * attended length of each sequence including this step's token, 1 <=
+ * seq_len <= max_pages*256.  plan: host int32 array of plan_capacity entries,
+ * filled with the plan (copy it to the device as is).  info receives the
+ * sizes, including the workspace bytes the decode/combine pair needs.
+ * KVQ_ESIZE if plan_capacity is too small (info->plan_len then holds the
+ * needed length). */
+typedef struct {
+    int32_t n_units;        /* work units = CTAs of the decode launch */
+    int32_t n_seq;
+    int32_t n_kv_heads;
+    int32_t group;          /* query heads per KV head */
+    int32_t plan_len;       /* int32 entries used in the plan array */
+    int32_t chunk_tokens;   /* largest unit, in tokens */
+    uint64_t workspace_bytes;
+} kvq_plan_info;
+
+int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len, int max_pages, int n_ctas,
+                    int32_t *plan, int plan_capacity, kvq_plan_info *info);
+
+/* paged_decode_attn_<fmt>: per work unit of the plan, single-token attention
+ * of the G query heads of one KV head over the unit's tokens, reading the
+ * quantised codes through the page table and dequantising inside the score
+ * and value loops ([Strata] "4-bit KV 缓存": scores on the rotated q and k,
+ * values mixed in the rotated space).  Scores are q.k_hat/16 with k_hat =
+ * (c-8)d (q4_0) or c d (int8); the softmax is online in fp32; all G heads of
+ * a group share one read of each K/V tile.  Writes, per unit, the unnormalised
+ * partial output and its running max and sum to the workspace.
+ *  q          device fp32 [n_seq][n_q_heads][256]; for q4_0 the output of
+ *             q_rotate, for int8 and k8v4 the plain query
+ *  page_table device int32 [n_seq][max_pages]
+ *  plan       device copy of the kvq_decode_plan array; info its host info
+ *  workspace  device, at least info->workspace_bytes
+ * The pool's format must match the entry point (KVQ_EINVAL otherwise). */
+int paged_decode_attn_int8(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                           int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                           uint64_t workspace_bytes, int32_t *status, void *stream);
+int paged_decode_attn_q4_0(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                           int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                           uint64_t workspace_bytes, int32_t *status, void *stream);
+int paged_decode_attn_k8v4(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                           int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                           uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* The same computation on CUDA cores only (fp32 FMA, no tensor cores).  Kept
+ * as the measured control for the tensor-core kernels above; fmt selects the
+ * format. */
+int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const float *q,
+                               const int32_t *page_table, int max_pages, const int32_t *plan,
+                               const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,
+                               int32_t *status, void *stream);
+
+/* attn_combine: for each (sequence, query head), merge the partials of its
+ * units with the log-sum-exp rule (M = max m_j, L = sum l_j 2^(m_j - M),
+ * o' = sum 2^(m_j - M) o_j / L), then, if inverse_fwht is non-zero (q4_0 and
+ * k8v4: V was stored rotated), apply H/16 once more ([Strata] "4-bit KV 缓存":
+ * H is its own inverse).  Writes out_bf16 (device uint16 bf16 bits
+ * [n_seq][n_q_heads][256], round to nearest even) and, if non-NULL, out_f32
+ * (device fp32, same shape). */
+int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,
+                 uint16_t *out_bf16, float *out_f32, void *stream);
+
+/* Library version string. */
+const char *kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,222 @@
+"""Python binding of the quantized paged decode-attention library (libkvq.so).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are PyTorch device tensors (memory and streams come from
+PyTorch); the library itself never allocates.  If the compiled library is
+missing, importing the binding's functions raises ``KVQError`` at once: there
+is no fallback implementation.
+
+Names follow the C ABI in ``include/kvq.h``: ``q_rotate``, ``kv_append``,
+``paged_decode_attn_{int8,q4_0,k8v4}``, ``attn_combine`` plus the host
+helpers ``pool_bytes``, ``pool_layout`` and ``decode_plan``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+INT8, Q4_0, K8V4 = 0, 1, 2
+FORMATS = {"int8": INT8, "q4_0": Q4_0, "k8v4": K8V4}
+HEAD_DIM = 256
+PAGE_TOKENS = 256
+
+STATUS_BAD_SLOT, STATUS_BAD_PLAN, STATUS_TIMEOUT = 1, 2, 4
+ERRORS = {-1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_EALIGN", -4: "KVQ_ECUDA", -5: "KVQ_ESIZE"}
+
+# entry points declared in include/kvq.h
+EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kvq_decode_plan",
+           "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
+           "paged_decode_attn_cudacore", "attn_combine"]
+
+
+class KVQError(RuntimeError):
+    pass
+
+
+class PoolDesc(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("n_pages", ctypes.c_int32),
+                ("fmt", ctypes.c_int32)]
+
+
+class Pool(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("desc", PoolDesc)]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("tile_bytes", "k_codes_off", "k_scales_off", "v_codes_off", "v_scales_off", "page_bytes",
+                 "head_stride", "slot_stride", "layer_stride", "total_bytes", "bytes_per_token_head")]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("n_units", ctypes.c_int32), ("n_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("group", ctypes.c_int32), ("plan_len", ctypes.c_int32), ("chunk_tokens", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libkvq.so (raises KVQError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise KVQError(f"{LIB_PATH} is missing: run `python -m quantized_kv_cache_17_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.kvq_version.restype = ctypes.c_char_p
+        L.kvq_pool_bytes.argtypes = [ctypes.POINTER(PoolDesc), ctypes.POINTER(ctypes.c_uint64)]
+        L.kvq_pool_layout.argtypes = [ctypes.POINTER(PoolDesc), ctypes.POINTER(Layout)]
+        L.q_rotate.argtypes = [P, P, I64, P]
+        L.kv_append.argtypes = [ctypes.POINTER(Pool), I32, P, P, I64, P, P, P, I32, I32, P, P]
+        L.kvq_decode_plan.argtypes = [ctypes.POINTER(PoolDesc), I32, P, I32, I32, P, I32, ctypes.POINTER(PlanInfo)]
+        dec = [ctypes.POINTER(Pool), I32, P, P, I32, P, ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P]
+        for n in ("paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4"):
+            getattr(L, n).argtypes = dec
+        L.paged_decode_attn_cudacore.argtypes = [I32] + dec
+        L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
+        for n in EXPORTS[1:]:
+            getattr(L, n).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise KVQError(f"{what} failed: {ERRORS.get(rc, rc)}")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_desc(n_layers: int, n_kv_heads: int, n_q_heads: int, n_pages: int, fmt) -> PoolDesc:
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    return PoolDesc(n_layers, n_kv_heads, n_q_heads, HEAD_DIM, PAGE_TOKENS, n_pages, f)
+
+
+def pool_bytes(desc: PoolDesc) -> int:
+    b = ctypes.c_uint64()
+    _check(lib().kvq_pool_bytes(ctypes.byref(desc), ctypes.byref(b)), "kvq_pool_bytes")
+    return b.value
+
+
+def pool_layout(desc: PoolDesc) -> Layout:
+    L = Layout()
+    _check(lib().kvq_pool_layout(ctypes.byref(desc), ctypes.byref(L)), "kvq_pool_layout")
+    return L
+
+
+@dataclass
+class KVPool:
+    """A pool descriptor plus the caller-owned device buffer that holds it."""
+    desc: PoolDesc
+    buf: object   # torch.uint8 device tensor of pool_bytes(desc) bytes
+
+    @staticmethod
+    def allocate(desc: PoolDesc, device="cuda"):
+        import torch
+        return KVPool(desc, torch.zeros(pool_bytes(desc), dtype=torch.uint8, device=device))
+
+    def c_pool(self) -> Pool:
+        return Pool(self.buf.data_ptr(), self.desc)
+
+    @property
+    def fmt(self) -> int:
+        return self.desc.fmt
+
+
+def q_rotate(q, out=None, stream=None):
+    """q_rot = (H/16) q for [..., 256] fp32 device tensors; out may alias q."""
+    if out is None:
+        out = q.new_empty(q.shape)
+    n = q.numel() // HEAD_DIM
+    _check(lib().q_rotate(_ptr(q), _ptr(out), n, _stream(stream)), "q_rotate")
+    return out
+
+
+def kv_append(pool: KVPool, layer: int, k, v, row_pos, page_table, row_seq=None, status=None, stream=None):
+    """Rotate/quantise/scatter rows k, v ([n_rows, n_kv_heads, 256] fp32)."""
+    n_rows = k.shape[0]
+    n_seq, max_pages = page_table.shape
+    cp = pool.c_pool()
+    _check(lib().kv_append(ctypes.byref(cp), layer, _ptr(k), _ptr(v), n_rows, _ptr(row_seq), _ptr(row_pos),
+                           _ptr(page_table), max_pages, n_seq, _ptr(status), _stream(stream)), "kv_append")
+
+
+def decode_plan(desc: PoolDesc, seq_lens: Sequence[int], max_pages: int, n_ctas: int = 0):
+    """Host split plan: returns (plan int32 numpy array, PlanInfo)."""
+    sl = np.ascontiguousarray(np.asarray(seq_lens, np.int32))
+    info = PlanInfo()
+    rc = lib().kvq_decode_plan(ctypes.byref(desc), len(sl), sl.ctypes.data, max_pages, n_ctas, None, 0,
+                               ctypes.byref(info))
+    if rc != -5:
+        _check(rc, "kvq_decode_plan")
+    plan = np.zeros(info.plan_len, np.int32)
+    _check(lib().kvq_decode_plan(ctypes.byref(desc), len(sl), sl.ctypes.data, max_pages, n_ctas,
+                                 plan.ctypes.data, len(plan), ctypes.byref(info)), "kvq_decode_plan")
+    return plan, info
+
+
+_DECODE = {INT8: "paged_decode_attn_int8", Q4_0: "paged_decode_attn_q4_0", K8V4: "paged_decode_attn_k8v4"}
+
+
+def paged_decode_attn(pool: KVPool, layer: int, q, page_table, plan_dev, info: PlanInfo, workspace, status=None,
+                      stream=None, cudacore: bool = False):
+    """Split-K decode attention of the pool's format (tensor-core kernel, or
+    the CUDA-core control when cudacore=True); partials go to workspace."""
+    cp = pool.c_pool()
+    args = (ctypes.byref(cp), layer, _ptr(q), _ptr(page_table), page_table.shape[1], _ptr(plan_dev),
+            ctypes.byref(info), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+            _stream(stream))
+    if cudacore:
+        _check(lib().paged_decode_attn_cudacore(pool.fmt, *args), "paged_decode_attn_cudacore")
+    else:
+        _check(getattr(lib(), _DECODE[pool.fmt])(*args), _DECODE[pool.fmt])
+
+
+def paged_decode_attn_int8(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
+    assert pool.fmt == INT8
+    paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def paged_decode_attn_q4_0(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
+    assert pool.fmt == Q4_0
+    paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def paged_decode_attn_k8v4(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
+    assert pool.fmt == K8V4
+    paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def attn_combine(workspace, plan_dev, info: PlanInfo, inverse_fwht: bool, out_bf16, out_f32=None, stream=None):
+    """Merge the partials; out_bf16 is a bf16 (or int16/uint16) tensor [n_seq, n_q_heads, 256]."""
+    _check(lib().attn_combine(_ptr(workspace), _ptr(plan_dev), ctypes.byref(info), 1 if inverse_fwht else 0,
+                              _ptr(out_bf16), _ptr(out_f32), _stream(stream)), "attn_combine")
+
+
+def rotated_v(fmt) -> bool:
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    return f in (Q4_0, K8V4)
+
+
+def rotated_q(fmt) -> bool:
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    return f == Q4_0

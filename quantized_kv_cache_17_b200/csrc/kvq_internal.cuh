@@ -1,0 +1,221 @@
+// Internal definitions shared by the CUDA translation units of the library:
+// pool layout constants, plan layout, and small PTX wrappers (mbarrier, bulk
+// copy, mma.sync, bounded waits).  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int D = 256;            // head_dim
+constexpr int PAGE = 256;         // tokens per page
+constexpr int TILE = 8;           // tokens per tile
+constexpr int TILES_PER_PAGE = PAGE / TILE;
+constexpr int STEP_TOKENS = 64;   // granularity of the split plan (one pipeline stage)
+constexpr int PLAN_HEADER = 8;
+constexpr int PLAN_MAGIC = 0x4B565131;  // "KVQ1"
+constexpr int WS_TAIL = 16;       // m[8], l[8] after o[G][256] in one workspace unit
+
+// ---------------------------------------------------------------------------
+// Pool layout.
+//
+// pool = [layer][slot][kv_head] page blocks; page block = 32 tiles of 8 tokens;
+// tile = [K codes | K scales | V codes | V scales].  Two kinds of part:
+//
+//   Q4 part (q4_0): codes 1024 B (8 tok x 256 x 4 bit), scales 128 B (8 tok x 8 fp16)
+//   I8 part (int8): codes 2048 B (8 tok x 256 x 8 bit), scales  64 B (8 tok x 4 fp16)
+//
+// Formats: INT8 = (K I8, V I8); Q4_0 = (K Q4, V Q4); K8V4 = (K I8, V Q4).
+//
+// Code arrangement inside a tile (r = token in tile 0..7).  Each is the
+// register-fragment order of mma.sync.m16n8k16 so that lane (g = lane/4,
+// t = lane%4) finds its operands in 16-byte words at lane*16 of 512-byte rows:
+//
+//  K side, Q4: 32-bit word W(r, b, j) (block b = 32 dims, j 0..3) at
+//      (b>>2)*512 + (r*4 + j)*16 + (b&3)*4; nibble n holds dim
+//      32b + 8(n&3) + (n>>2) + 2j.
+//  V side, Q4: word W(p, b, g) (token pair p: tokens 2p, 2p+1; g 0..7) at
+//      (b>>2)*512 + (g*4 + p)*16 + (b&3)*4; nibble n holds token 2p + (n>>2),
+//      dim 32b + g + 8(n&3).
+//  K side, I8: word W(r, s, j) (k-step s = 16 dims) at
+//      (s>>2)*512 + (r*4 + j)*16 + (s&3)*4; byte n holds dim 16s + 2j + {0,1,8,9}[n].
+//  V side, I8: word W(p, m, g) (m-tile m = 16 dims) at
+//      (m>>2)*512 + (g*4 + p)*16 + (m&3)*4; byte n holds token 2p + (n&1),
+//      dim 16m + g + 8(n>>1).
+//  Scales (fp16): Q4 token r, block b at (r>>1)*32 + b*4 + (r&1)*2;
+//                 I8 token r, group q at (r>>1)*16 + q*4 + (r&1)*2.
+// int8 codes are stored as two's complement bytes.
+// ---------------------------------------------------------------------------
+enum Part : int { PART_Q4 = 0, PART_I8 = 1 };
+
+__host__ __device__ constexpr int part_code_bytes(int p) { return p == PART_Q4 ? 1024 : 2048; }
+__host__ __device__ constexpr int part_scale_bytes(int p) { return p == PART_Q4 ? 128 : 64; }
+
+template <int FMT> struct Fmt;
+template <> struct Fmt<KVQ_INT8> {
+    static constexpr int KP = PART_I8, VP = PART_I8;
+    static constexpr bool KROT = false, VROT = false;
+};
+template <> struct Fmt<KVQ_Q4_0> {
+    static constexpr int KP = PART_Q4, VP = PART_Q4;
+    static constexpr bool KROT = true, VROT = true;
+};
+template <> struct Fmt<KVQ_K8V4> {
+    static constexpr int KP = PART_I8, VP = PART_Q4;
+    static constexpr bool KROT = false, VROT = true;
+};
+
+template <int FMT> struct TileLayout {
+    static constexpr int KP = Fmt<FMT>::KP, VP = Fmt<FMT>::VP;
+    static constexpr int KC = 0;
+    static constexpr int KS = KC + part_code_bytes(KP);
+    static constexpr int VC = KS + part_scale_bytes(KP);
+    static constexpr int VS = VC + part_code_bytes(VP);
+    static constexpr int BYTES = VS + part_scale_bytes(VP);
+    static constexpr int PAGE_BYTES = BYTES * TILES_PER_PAGE;
+};
+
+inline int host_part_k(int fmt) { return fmt == KVQ_Q4_0 ? PART_Q4 : PART_I8; }
+inline int host_part_v(int fmt) { return fmt == KVQ_INT8 ? PART_I8 : PART_Q4; }
+
+struct PoolGeom {
+    int64_t layer_stride, slot_stride, page_bytes;
+    int n_pages, n_kv_heads;
+};
+
+// ---------------------------------------------------------------------------
+// Plan (int32): [magic, n_units, n_seq, n_kv_heads, group, chunk, 0, 0]
+//               units[n_units][4] = {seq, kv_head, t_begin, t_end}
+//               start[n_seq * n_kv_heads + 1]  (first unit of each (seq, kv head))
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int plan_len_for(int n_units, int n_seq, int n_kv) {
+    return PLAN_HEADER + 4 * n_units + n_seq * n_kv + 1;
+}
+__host__ __device__ inline int ws_unit_floats(int G) { return G * D + WS_TAIL; }
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait on an mbarrier phase with a time limit.  Returns false (and the caller
+// records KVQ_STATUS_TIMEOUT) if the phase did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier.
+// src, dst 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint4 lds128(const void *p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));  // (a & b) | c
+    return d;
+}
+
+// D = A * B + C, m16n8k16, fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void status_or(int32_t *status, uint32_t bits) {
+    if (status) atomicOr(reinterpret_cast<unsigned int *>(status), bits);
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
+    return *reinterpret_cast<__half2 *>(&u);
+}
+
+// Host launchers (defined in the .cu files).
+cudaError_t launch_q_rotate(const float *q, float *q_rot, int64_t n_vec, cudaStream_t s);
+cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer, const float *k,
+                          const float *v, int64_t n_rows, const int32_t *row_seq, const int32_t *row_pos,
+                          const int32_t *page_table, int max_pages, int n_seq, int32_t *status, cudaStream_t s);
+cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
+                          const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
+                          const kvq_plan_info &info, float *ws, int32_t *status, cudaStream_t s);
+cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_info &info, int inverse_fwht,
+                           uint16_t *out_bf16, float *out_f32, cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,188 @@
+"""GPU vs oracle parity at sizes the oracle finishes in seconds.
+
+Bit-exact: the device generator against numpy, q_rotate and the codes and
+fp16 scales written by kv_append.  Within the tolerance (fp32 output vs the
+fp64 oracle on the GPU's own codes: relative L2 <= 1e-3 per output vector and
+max-abs <= 2e-3): decode + combine for every format, on both the tensor-core
+kernels and the CUDA-core control, across several tiles, pages, ragged tails,
+split counts, group sizes and permuted page tables.  All calls go through the
+C ABI (via the ctypes binding).
+"""
+import numpy as np
+import pytest
+import torch
+
+import kvq_inputs
+import oracle
+import quantized_kv_cache_17_b200 as kvq
+from kvq_inputs import device as kdev
+from tests import gpu_common as gc
+from tests import kvq_layout
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from quantized_kv_cache_17_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def small(fmt, Hq, Hkv, seq_lens, order="permuted", outlier="mul20", q_post=1.0, q_outliers=True, n_out=4,
+          layers=1, name=None):
+    return kvq_inputs.Workload(name=name or f"small_{fmt}_{Hq}_{Hkv}_{'_'.join(map(str, seq_lens))}", index=9,
+                               fmt=fmt, n_layers=layers, n_q_heads=Hq, n_kv_heads=Hkv, seq_lens=list(seq_lens),
+                               page_order=order, n_outlier=n_out, outlier_kind=outlier, q_post=q_post,
+                               q_outliers=q_outliers)
+
+
+# ---------------------------------------------------------------------------
+def test_device_generator_bit_exact():
+    w = kvq_inputs.workload("qwen27b_q4_0_262k")
+    for tab, key, row0 in [(w.kv_table(3), w.k_key(3, 0), 262000), (w.q_table(1), w.q_key(1, 0), 0),
+                           (kvq_inputs.workload("tiny_q4_0_1k").kv_table(0), 12345, 17),
+                           (kvq_inputs.workload("qwen27b_int8_32k").kv_table(0), 999, 5)]:
+        dt = kdev.DeviceTable(tab)
+        got = kdev.gen_rows_device(key, dt, row0, 37).cpu().numpy()
+        want = kvq_inputs.gen_rows(key, tab, row0, 37)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("n_vec", [1, 3, 24, 1000])
+def test_q_rotate_bit_exact(n_vec):
+    w = kvq_inputs.workload("tiny_q4_0_1k")
+    qh = kvq_inputs.gen_rows(77, w.q_table(0), 0, n_vec).reshape(-1, 256)[:n_vec].copy()
+    q = torch.from_numpy(qh).cuda()
+    got = kvq.q_rotate(q).cpu().numpy()
+    want = oracle.fwht256_f32(qh)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    kvq.q_rotate(q, out=q)            # in place
+    assert np.array_equal(q.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+def test_kv_append_bit_exact(fmt):
+    w = small(fmt, 12, 2, [700, 1025], outlier="student_t", n_out=8)
+    dw = kdev.build_pool(w, extra_slots=3, prefill_last=True)
+    for b, T in enumerate(w.seq_lens):
+        for g in range(w.n_kv_heads):
+            kc, ks, vc, vs = gc.pool_codes(dw, 0, b, g)
+            k = w.k_rows(0, b, 0, T)[:, g]
+            v = w.v_rows(0, b, 0, T)[:, g]
+            okc, oks, ovc, ovs = oracle.append_rows(fmt, k, v)
+            assert np.array_equal(kc, okc) and np.array_equal(ks, oks)
+            assert np.array_equal(vc, ovc) and np.array_equal(vs, ovs)
+
+
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+def test_kv_append_single_rows_match_batch(fmt):
+    """Decode-style appends (one row per sequence per call) give the same bytes."""
+    w = small(fmt, 8, 2, [40, 300])
+    a = kdev.build_pool(w, prefill_last=True)
+    bpool = kdev.build_pool(w, prefill_last=False)
+    _, k, v, pos = kdev.step_inputs(w, [0])
+    kvq.kv_append(bpool.pool, 0, k[0], v[0], pos, bpool.page_table)
+    torch.cuda.synchronize()
+    layout = kvq.pool_layout(a.pool.desc)
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            x = kvq_layout.gather_sequence(fmt, a.pool.buf, layout, 0, g, a.page_table_host[b], w.seq_lens[b])
+            y = kvq_layout.gather_sequence(fmt, bpool.pool.buf, layout, 0, g, bpool.page_table_host[b],
+                                           w.seq_lens[b])
+            for p, r in zip(x, y):
+                assert np.array_equal(p, r)
+
+
+def test_kv_append_bad_slot_sets_status():
+    w = small("q4_0", 4, 1, [300])
+    dw = kdev.build_pool(w)
+    pt = dw.page_table.clone()
+    pt[0, 1] = 10_000                     # outside the pool: the row must be skipped, not written
+    before = dw.pool.buf.clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    k = torch.randn(1, 1, 256, device="cuda")
+    kvq.kv_append(dw.pool, 0, k, k, torch.tensor([299], dtype=torch.int32, device="cuda"), pt, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & kvq.STATUS_BAD_SLOT
+    assert torch.equal(before, dw.pool.buf)
+
+
+# ---------------------------------------------------------------------------
+CASES = {
+    # name: (workload, n_ctas values)
+    "tiny_1k": (kvq_inputs.workload("tiny_q4_0_1k"), [0, 3]),
+    "cross_page_1025": (kvq_inputs.scaled(kvq_inputs.workload("tiny_q4_0_1k"), [1025]), [0, 1]),
+    "ragged_g6": (small("q4_0", 24, 4, [1, 77, 300, 1025], outlier="student_t", q_post=1 / 16,
+                        q_outliers=False, n_out=8), [0, 5]),
+    "ragged_g8": (small("q4_0", 16, 2, [513, 64, 8]), [0, 2]),
+}
+
+
+def _case(name, fmt):
+    w, nctas = CASES[name]
+    if fmt != w.fmt:
+        import dataclasses
+        w = dataclasses.replace(w, fmt=fmt, name=w.name + "_" + fmt)
+    return w, nctas
+
+
+@pytest.mark.parametrize("impl", ["mma", "alu"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("case", list(CASES))
+def test_decode_matches_oracle(case, fmt, impl):
+    w, nctas = _case(case, fmt)
+    dw = kdev.build_pool(w, extra_slots=2)
+    q, k, v, pos = kdev.step_inputs(w, [0])
+    kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table)          # this step's token
+    refs = {}
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            refs[b, g] = gc.oracle_group(dw, 0, b, g)
+    for n_ctas in nctas:
+        out_f, out_bf, status, plan, info = gc.decode_step(dw, 0, q[0], impl=impl, n_ctas=n_ctas)
+        assert status == 0
+        G = w.group
+        for (b, g), ref in refs.items():
+            gc.assert_close(out_f[b, g * G:(g + 1) * G], ref, f"{case}/{fmt}/{impl}/nctas={n_ctas} b={b} g={g}")
+        ref_all = np.stack([np.concatenate([refs[b, g] for g in range(w.n_kv_heads)]) for b in range(w.batch)])
+        gc.assert_bf16_consistent(out_f, out_bf, ref_all)
+
+
+def test_decode_single_token_context():
+    """T = 1: the output is that token's dequantised value, un-rotated."""
+    w = small("q4_0", 6, 1, [1])
+    dw = kdev.build_pool(w)
+    q, k, v, pos = kdev.step_inputs(w, [0])
+    kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table)
+    out_f, _, status, _, _ = gc.decode_step(dw, 0, q[0])
+    kc, ks, vc, vs = gc.pool_codes(dw, 0, 0, 0)
+    vhat = oracle.fwht256_f64(oracle.dequant_rows(True, vc, vs))[0]
+    for h in range(6):
+        gc.assert_close(out_f[0, h], vhat, "T=1")
+    assert status == 0
+
+
+def test_decode_bad_page_slot_reports_status():
+    w = small("q4_0", 4, 1, [600])
+    dw = kdev.build_pool(w, prefill_last=True)
+    dw.page_table[0, 1] = -7
+    q, _, _, _ = kdev.step_inputs(w, [0])
+    out_f, _, status, _, _ = gc.decode_step(dw, 0, q[0])
+    assert status & kvq.STATUS_BAD_SLOT
+    assert np.isfinite(out_f).all()
+
+
+def test_decode_bad_plan_reports_status():
+    w = small("int8", 4, 1, [300])
+    dw = kdev.build_pool(w, prefill_last=True)
+    plan, info = kvq.decode_plan(dw.pool.desc, dw.seq_lens, dw.page_table.shape[1], 0)
+    plan[8 + 2] = 32            # unit start not on a 64-token step
+    plan_d = torch.from_numpy(plan).cuda()
+    ws = torch.empty(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, _, _, _ = kdev.step_inputs(w, [0])
+    kvq.paged_decode_attn(dw.pool, 0, q[0], dw.page_table, plan_d, info, ws, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & kvq.STATUS_BAD_PLAN
