@@ -209,44 +209,68 @@ def run_ours(args):
     q, k_new, v_new, pos = kdev.step_inputs(w, list(range(L)))
     plan, info = kvq.decode_plan(dw.pool.desc, w.seq_lens, dw.page_table.shape[1], args.n_ctas)
     plan_d = torch.from_numpy(plan).cuda()
-    ws = torch.empty(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
     q_rot = torch.empty_like(q)
     out_bf = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
     out_f = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
     rot_q, rot_v = kvq.rotated_q(fmt), kvq.rotated_v(fmt)
     use_alu = args.decode == "alu"
+    fused = not use_alu and not args.no_fuse
     layout = kvq.pool_layout(dw.pool.desc)
     kv_bytes_layer = sum(w.seq_lens) * w.n_kv_heads * layout.bytes_per_token_head
 
-    def layer_step(l, dec_events=None):
+    def layer_step(l):
         qq = q[l]
         if rot_q:
-            kvq.q_rotate(qq, q_rot[l], stream)
+            kvq.q_rotate(qq, q_rot[l])
             qq = q_rot[l]
-        kvq.kv_append(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, status=status, stream=stream)
-        if dec_events is not None:
-            dec_events[0].record(stream)
-        kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, stream, cudacore=use_alu)
-        if dec_events is not None:
-            dec_events[1].record(stream)
-        kvq.attn_combine(ws, plan_d, info, rot_v, out_bf[l], out_f[l], stream)
+        kvq.kv_append(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, status=status)
+        if fused:
+            kvq.paged_decode_attn_combined(dw.pool, l, qq, dw.page_table, plan_d, info, ws, out_bf[l], out_f[l],
+                                           status)
+        else:
+            kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, cudacore=use_alu)
+            kvq.attn_combine(ws, plan_d, info, rot_v, out_bf[l], out_f[l])
 
-    def step(evs=None):
+    def step():
         for l in range(L):
-            layer_step(l, evs[l] if evs is not None else None)
+            layer_step(l)
 
-    launches_per_layer = 3 + (1 if rot_q else 0)
+    def decode_only():
+        for l in range(L):
+            qq = q_rot[l] if rot_q else q[l]
+            if fused:
+                kvq.paged_decode_attn_combined(dw.pool, l, qq, dw.page_table, plan_d, info, ws, out_bf[l], out_f[l],
+                                               status)
+            else:
+                kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, cudacore=use_alu)
+
+    launches_per_layer = (2 if fused else 3) + (1 if rot_q else 0)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
+    # eager warm-up (sets kernel attributes, fills caches of the runtime), then
+    # capture one whole step and the decode launches alone as CUDA graphs
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0, f"kernel status {status.item()}"
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g_step, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_step, stream=cap):
+            step()
+        with torch.cuda.graph(g_dec, stream=cap):
+            decode_only()
+    torch.cuda.current_stream().wait_stream(cap)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        g_step.replay()
+    torch.cuda.synchronize()
 
     uuid = ""
     try:
@@ -254,8 +278,6 @@ def run_ours(args):
     except Exception:
         pass
     sampler = ClockSampler(uuid)
-    dec_evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
-               for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.start()
     time.sleep(0.3)
@@ -263,16 +285,26 @@ def run_ours(args):
     torch.cuda.synchronize()
     torch.cuda.cudart().cudaProfilerStart()      # an ncu launch list with --profile-from-start off sees only this region
     t_start.record(stream)
-    for s in range(args.steps):
-        step(dec_evs[s])
+    for _ in range(args.steps):
+        g_step.replay()
     t_end.record(stream)
     torch.cuda.synchronize()
     torch.cuda.cudart().cudaProfilerStop()
     barrier()
     clocks = sampler.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
-    dec_ms = [e[0].elapsed_time(e[1]) for st in dec_evs for e in st]
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+
+    # the decode kernel alone: back-to-back launches of all layers, CUDA events on
+    # the launching stream around the replays
+    d_start, d_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g_dec.replay()
+    torch.cuda.synchronize()
+    d_start.record(stream)
+    for _ in range(args.steps):
+        g_dec.replay()
+    d_end.record(stream)
+    torch.cuda.synchronize()
+    dec_avg_ms = d_start.elapsed_time(d_end) / (args.steps * L)
 
     # ---- end to end: host buffers, copies inside the timed region ---------------
     q_h = q.cpu().pin_memory()
@@ -289,13 +321,14 @@ def run_ours(args):
         q.copy_(q_h, non_blocking=True)
         k_new.copy_(k_h, non_blocking=True)
         v_new.copy_(v_h, non_blocking=True)
-        step()
+        g_step.replay()
         o_h.copy_(out_bf, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
     assert int(status.item()) == 0, f"kernel status {status.item()}"
+    del g_step, g_dec
 
     if dist is not None:
         t = torch.tensor([elapsed_ms, e2e_ms, dec_avg_ms], dtype=torch.float64, device="cuda")
@@ -309,7 +342,7 @@ def run_ours(args):
     tok_s = world * w.batch / (ms_per_step * 1e-3)
     peak, peak_kind = peaks()
     achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
-    kernel_tag = "decode_alu" if use_alu else "decode_mma"
+    kernel_tag = "decode_alu" if use_alu else ("decode_mma_fused" if fused else "decode_mma")
     traffic = ncu_traffic(kernel_tag, w.name)
 
     cpu = None
@@ -354,6 +387,7 @@ def run_ours(args):
                 "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
                 "gpu_launches": args.steps * L * launches_per_layer,
+                "launch": "CUDA graph of the 16-layer step",
                 "clocks": clocks,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
@@ -371,6 +405,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--decode", default="mma", choices=["mma", "alu"])
     ap.add_argument("--n-ctas", type=int, default=0)
+    ap.add_argument("--no-fuse", action="store_true", help="separate attn_combine launch")
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-groups", type=int, default=4)

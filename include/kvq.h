@@ -173,7 +173,10 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
  *             q_rotate, for int8 and k8v4 the plain query
  *  page_table device int32 [n_seq][max_pages]
  *  plan       device copy of the kvq_decode_plan array; info its host info
- *  workspace  device, at least info->workspace_bytes
+ *  workspace  device, at least info->workspace_bytes; it ends with one int32
+ *             arrival counter per (sequence, KV head) group that the
+ *             *_combined entry points use: zero-fill the workspace once before
+ *             its first use with them (every call leaves the counters at zero)
  * The pool's format must match the entry point (KVQ_EINVAL otherwise). */
 int paged_decode_attn_int8(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                            int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
@@ -184,6 +187,25 @@ int paged_decode_attn_q4_0(const kvq_pool *pool, int layer, const float *q, cons
 int paged_decode_attn_k8v4(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                            int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                            uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* paged_decode_attn_<fmt>_combined: the same decode with attn_combine fused
+ * into it.  The last CTA to finish a (sequence, KV head) group (counted with an
+ * atomic counter in the workspace, never a wait) merges the group's partials,
+ * un-rotates (q4_0, k8v4) and writes out_bf16 / out_f32 exactly as
+ * attn_combine would.  Saves the combine launch; otherwise identical contract.
+ * Calls on the same workspace must not overlap on the GPU. */
+int paged_decode_attn_int8_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                    int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                                    uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
+                                    void *stream);
+int paged_decode_attn_q4_0_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                    int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                                    uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
+                                    void *stream);
+int paged_decode_attn_k8v4_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                    int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                                    uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
+                                    void *stream);
 
 /* The same computation on CUDA cores only (fp32 FMA, no tensor cores).  Kept
  * as the measured control for the tensor-core kernels above; fmt selects the

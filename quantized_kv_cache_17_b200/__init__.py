@@ -33,6 +33,7 @@ ERRORS = {-1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_EALIGN", -4: "KVQ_E
 # entry points declared in include/kvq.h
 EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kvq_decode_plan",
            "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
+           "paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined", "paged_decode_attn_k8v4_combined",
            "paged_decode_attn_cudacore", "attn_combine"]
 
 
@@ -82,6 +83,9 @@ def lib():
         dec = [ctypes.POINTER(Pool), I32, P, P, I32, P, ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P]
         for n in ("paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4"):
             getattr(L, n).argtypes = dec
+        for n in ("paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined",
+                  "paged_decode_attn_k8v4_combined"):
+            getattr(L, n).argtypes = dec[:-2] + [P, P] + dec[-2:]
         L.paged_decode_attn_cudacore.argtypes = [I32] + dec
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
         for n in EXPORTS[1:]:
@@ -175,6 +179,18 @@ def decode_plan(desc: PoolDesc, seq_lens: Sequence[int], max_pages: int, n_ctas:
 
 
 _DECODE = {INT8: "paged_decode_attn_int8", Q4_0: "paged_decode_attn_q4_0", K8V4: "paged_decode_attn_k8v4"}
+
+
+def paged_decode_attn_combined(pool: KVPool, layer: int, q, page_table, plan_dev, info: PlanInfo, workspace,
+                               out_bf16, out_f32=None, status=None, stream=None):
+    """Decode with the combine fused in; workspace must have been zero-filled
+    once before its first use (the call leaves its counters at zero)."""
+    cp = pool.c_pool()
+    name = _DECODE[pool.fmt] + "_combined"
+    _check(getattr(lib(), name)(ctypes.byref(cp), layer, _ptr(q), _ptr(page_table), page_table.shape[1],
+                                _ptr(plan_dev), ctypes.byref(info), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _ptr(out_bf16), _ptr(out_f32),
+                                _ptr(status), _stream(stream)), name)
 
 
 def paged_decode_attn(pool: KVPool, layer: int, q, page_table, plan_dev, info: PlanInfo, workspace, status=None,

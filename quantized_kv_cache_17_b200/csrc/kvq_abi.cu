@@ -62,7 +62,8 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ECUDA; }
 
 int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                   int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
-                  uint64_t workspace_bytes, int32_t *status, void *stream) {
+                  uint64_t workspace_bytes, int32_t *status, void *stream, uint16_t *out_bf16 = nullptr,
+                  float *out_f32 = nullptr) {
     PoolGeom geo;
     int rc = check_pool(pool, layer, &geo);
     if (rc) return rc;
@@ -74,8 +75,12 @@ int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float
         return KVQ_EINVAL;
     if ((int64_t)max_pages * PAGE > INT32_MAX) return KVQ_EINVAL;
     if (workspace_bytes < info->workspace_bytes) return KVQ_ESIZE;
+    if ((out_bf16 && !aligned16(out_bf16)) || (out_f32 && !aligned16(out_f32))) return KVQ_EALIGN;
+    if (!out_bf16 && out_f32) return KVQ_EINVAL;
+    const int inverse = fmt == KVQ_INT8 ? 0 : 1;
     return cuda_rc(launch_decode(fmt, tc, static_cast<const uint8_t *>(pool->base), geo, layer, q, page_table,
-                                 max_pages, plan, *info, workspace, status, static_cast<cudaStream_t>(stream)));
+                                 max_pages, plan, *info, workspace, status, inverse, out_bf16, out_f32,
+                                 static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -165,7 +170,7 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
     info->group = G;
     info->plan_len = len;
     info->chunk_tokens = (int32_t)(c * STEP_TOKENS);
-    info->workspace_bytes = (uint64_t)n_units * ws_unit_floats(G) * sizeof(float);
+    info->workspace_bytes = ws_bytes_for((int)n_units, G, n_seq * n_kv);
     if (!plan || plan_capacity < len) return KVQ_ESIZE;
     plan[0] = PLAN_MAGIC;
     plan[1] = (int32_t)n_units;
@@ -230,6 +235,19 @@ int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const f
     return decode_common(fmt, false, pool, layer, q, page_table, max_pages, plan, info, workspace, workspace_bytes,
                          status, stream);
 }
+
+#define KVQ_COMBINED(NAME, FMT)                                                                                 \
+    int NAME(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table, int max_pages,              \
+             const int32_t *plan, const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,             \
+             uint16_t *out_bf16, float *out_f32, int32_t *status, void *stream) {                                    \
+        if (!out_bf16) return KVQ_EINVAL;                                                                            \
+        return decode_common(FMT, true, pool, layer, q, page_table, max_pages, plan, info, workspace,               \
+                             workspace_bytes, status, stream, out_bf16, out_f32);                                   \
+    }
+KVQ_COMBINED(paged_decode_attn_int8_combined, KVQ_INT8)
+KVQ_COMBINED(paged_decode_attn_q4_0_combined, KVQ_Q4_0)
+KVQ_COMBINED(paged_decode_attn_k8v4_combined, KVQ_K8V4)
+#undef KVQ_COMBINED
 
 int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,
                  uint16_t *out_bf16, float *out_f32, void *stream) {

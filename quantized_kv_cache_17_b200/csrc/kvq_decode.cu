@@ -1,55 +1,46 @@
 // paged_decode_attn_{int8,q4_0,k8v4}: split-K single-token attention over the
-// quantised, paged KV cache, one CTA per work unit of the plan.
+// quantised, paged KV cache, one CTA per work unit of the plan; attn_combine:
+// the merge of a (sequence, KV head) group's partials, either as its own
+// launch or fused into the last CTA of the group.
 //
 // [Strata] "4-bit KV 缓存：先旋转，再压到 4-bit": scores are taken on the rotated
 // query and rotated keys (<Hq, Hk> = <q, k>), values are mixed in the rotated
-// space and the output is rotated back afterwards (attn_combine).  [Guide]
-// "一": 24 query heads share 4 KV heads (groups of 6), so every K/V tile read
-// from HBM serves the whole group.
+// space and the merged output is rotated back (H/16 is its own inverse).
+// [Guide] "一": 24 query heads share 4 KV heads (groups of 6), so every K/V
+// tile read from HBM serves the whole group.
 //
-// CTA = 8 consumer warps + 1 producer warp.  The producer streams the unit's
-// tokens in 64-token steps (8 tiles, contiguous inside one page block) with
-// 1-D bulk copies into a ring of shared-memory stages (full/empty mbarriers);
-// consumer warp w takes tile w of every step.  Each warp keeps its own online
-// softmax state; at the end the warps are merged in shared memory and the CTA
-// writes one partial (o[G][256] unnormalised, m[G], l[G], scores in log2 units).
+// Data path (both kernels): a copy warp streams the unit's tokens in 64-token
+// steps (8 tiles, contiguous inside one page block) with 1-D bulk copies into
+// a ring of shared-memory stages guarded by full/empty mbarriers.  At the end
+// the CTA merges its warps' softmax states in shared memory and writes one
+// partial (o[G][256] unnormalised, m[8], l[8]; scores in log2 units); with the
+// combine fused in, the last CTA of each (sequence, KV head) merges the group.
 //
-// Two compute policies share the scaffold:
-//  MmaCompute  - tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32).  Codes
-//                are exact in fp16; the query and the probabilities are split
-//                into fp16 hi + lo parts so the products keep ~22 bits.
-//                QK^T: rows = [8 heads hi | 8 heads lo], cols = 8 tokens,
-//                k = 16 dims; the per-block K scale is applied to the fp32
-//                block sums.  PV: rows = 16 dims, cols = 8 heads, k = [8 tokens
-//                hi-P | same 8 tokens lo-P]; the per-block V scale is folded
-//                into P before the split.  The score fragment of QK^T is exactly
-//                the P fragment PV needs, so no data moves between lanes.
-//  AluCompute  - the same computation with fp32 FMAs on CUDA cores only; the
-//                measured control for the tensor-core version.
+// Tensor-core kernel (the product), warp-specialised:
+//  - QK warps: the query of the group as mma.sync m16n8k16 A fragments in
+//    registers (rows = [8 heads, fp16 hi | same 8 heads, fp16 lo], k = 16
+//    dims), K codes unpacked to fp16 in registers as B (cols = 8 tokens),
+//    the per-block K scale applied to the fp32 block sums; online softmax;
+//    hands p (and the rescale factor of each head) to its PV warp through a
+//    small shared-memory ring.
+//  - PV warps: the output accumulators o[dims][heads] in registers; rows = 16
+//    dims of V codes (exact in fp16), k = [8 tokens with P'hi | the same 8
+//    tokens with P'lo], P' = p * dV formed as an exact fp16 pair.  The score
+//    fragment layout of QK is exactly the P fragment layout PV needs.
+//  - a scale warp converts each stage's fp16 K scales to fp32 once.
+// CUDA-core kernel (the measured control): the same computation with fp32
+// FMAs only.
+#include <type_traits>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr int NW = 8;                         // consumer warps
-constexpr int NTHREADS = (NW + 1) * 32;
 constexpr float QSCALE = 0.09016844005556021f;  // log2(e) / sqrt(256)
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-
-template <int FMT> struct Stages { static constexpr int N = 4; };
-template <> struct Stages<KVQ_Q4_0> { static constexpr int N = 5; };
-template <> struct Stages<KVQ_INT8> { static constexpr int N = 3; };
-template <> struct Stages<KVQ_K8V4> { static constexpr int N = 4; };
-
-template <int FMT> struct Smem {
-    static constexpr int STAGE_BYTES = NW * TileLayout<FMT>::BYTES;
-    static constexpr int NS = Stages<FMT>::N;
-    static constexpr int RING = NS * STAGE_BYTES;
-    static constexpr int MERGE = (8 * D + 2 * NW * 8 + 2 * 8) * 4;   // o[8][256], m/l per warp, M/L
-    static constexpr int DATA = RING > MERGE ? RING : MERGE;
-    static constexpr int BAR_OFF = (DATA + 15) & ~15;
-    static constexpr int TOTAL = BAR_OFF + NS * 16 + NS * 4 + 16;
-};
+constexpr int COMBINE_MAX_UNITS = 256;            // units per group merged in one pass of the combine
+constexpr int COMBINE_SMEM = 8 * D + 2 * 8 * COMBINE_MAX_UNITS + 16;   // floats of combine scratch
 
 __device__ __forceinline__ __half2 q4_lo_pair(uint32_t w) {     // nibbles 0 / 4 of each half -> c - 8
     return __hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(0x64086408u));
@@ -70,159 +61,319 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
     lo = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
 }
 
+// D = A * B (C = 0), A fragment from a 16-byte shared-memory word.
+__device__ __forceinline__ void mma_z(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "f"(0.f));
+}
+// D = A * B + D
+__device__ __forceinline__ void mma_acc(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ float4 lds128f(const float *p) {
+    const uint4 v = lds128(p);
+    return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+// (v0, v1) = 8 floats; pair i = floats 2i, 2i+1
+__device__ __forceinline__ float2 f2_at(const float4 &v0, const float4 &v1, int i) {
+    return i == 0 ? make_float2(v0.x, v0.y)
+                  : (i == 1 ? make_float2(v0.z, v0.w) : (i == 2 ? make_float2(v1.x, v1.y) : make_float2(v1.z, v1.w)));
+}
+__device__ __forceinline__ uint2 lds64(const void *p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+    return v;
+}
+__device__ __forceinline__ void sts128(void *p, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// Tensor-core compute policy
+// Tensor-core kernel: configuration
 // ---------------------------------------------------------------------------
-template <int FMT> struct MmaCompute {
+#ifndef KVQ_QK_WARPS
+#define KVQ_QK_WARPS 7       // QK warps per CTA (and as many PV warps)
+#endif
+
+template <int FMT> struct TcCfg {
     using L = TileLayout<FMT>;
-    uint32_t qa[16][4];
-    float o[16][4];
-    float m_run, l_run;
+    static constexpr int NQK = KVQ_QK_WARPS;
+    static constexpr int SCALE_WARP = 2 * NQK;
+    static constexpr int COPY_WARP = 2 * NQK + 1;
+    static constexpr int NTHREADS = (2 * NQK + 2) * 32;
+    static constexpr int ITEMS_PER_STAGE = 4;                   // an item = 2 tiles = 16 tokens
+    static constexpr int STAGE_BYTES = 8 * L::BYTES;
+    static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
+    static constexpr int DP = 4;                                // slots of each QK -> PV ring
+    // fp32 K scales of a stage: per tile, token pair t at float t*KSTRIDE (block
+    // or group j of tokens 2t, 2t+1 at 2j, 2j+1); the stride pads rows so the
+    // four pairs fall into different banks
+    static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
+    static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
+    static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
+    static constexpr int PSLOT = 32 * 4 + 8;                    // floats: p of 32 lanes x 4, alpha[8]
+    static constexpr int RING = NS * STAGE_BYTES;
+    static constexpr int MERGE = (COMBINE_SMEM > 8 * D + 2 * NQK * 8 + 16 ? COMBINE_SMEM : 8 * D + 2 * NQK * 8 + 16) * 4;
+    static constexpr int DATA = RING > MERGE ? RING : MERGE;
+    static constexpr int SFOFF = (DATA + 127) & ~127;
+    static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
+    static constexpr int BAR_OFF = POFF + NQK * DP * PSLOT * 4;
+    // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]
+    static constexpr int TOTAL = BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 16;
+    static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+};
+
+// Scale warp: convert the fp16 K scales of one stage (8 tiles) to fp32 rows.
+template <int FMT>
+__device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float *sf, int lane) {
+    using L = TileLayout<FMT>;
+    constexpr int KSB = part_scale_bytes(L::KP);        // fp16 bytes per tile: 4 token pairs
+    constexpr int PAIR_B = KSB / 4;                     // 32 (q4) or 16 (i8) bytes per pair
+    constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
+    constexpr int CPT = KSB / 16;                       // 16-byte chunks per tile
+    for (int c = lane; c < 8 * CPT; c += 32) {
+        const int tile = c / CPT, o = (c % CPT) * 16;
+        const int pair = o / PAIR_B, within = (o % PAIR_B) / 2;
+        const uint4 h = lds128(stage + tile * L::BYTES + L::KS + o);
+        float *dst = sf + tile * 4 * KSTRIDE + pair * KSTRIDE + within;
+        const float2 a = __half22float2(u32_as_h2(h.x)), b = __half22float2(u32_as_h2(h.y));
+        const float2 cc = __half22float2(u32_as_h2(h.z)), d = __half22float2(u32_as_h2(h.w));
+        sts128(dst, make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y)));
+        sts128(dst + 4, make_uint4(__float_as_uint(cc.x), __float_as_uint(cc.y), __float_as_uint(d.x), __float_as_uint(d.y)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// QK warp: scores and online softmax for one work item (tiles A, B = 16 tokens)
+// ---------------------------------------------------------------------------
+template <int FMT> struct QkWarp {
+    using L = TileLayout<FMT>;
+    using C = TcCfg<FMT>;
+    uint4 qa[16];          // A fragments of the 16 k-steps
+    float m_run, l_run;    // head g (the four lanes of a group agree)
+
+    // Fragment of k-step ks for lane (g, t): rows g (hi) / g+8 (lo) of head g,
+    // dims 16ks + 2t, +1 (a0/a1) and 16ks + 2t + 8, +9 (a2/a3).
+    __device__ static uint4 make_qfrag(const float *qg, int G, int ks, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (g < G) {
+            const float *p = qg + g * D + 16 * ks + 2 * t;
+            x[0] = p[0] * QSCALE; x[1] = p[1] * QSCALE; x[2] = p[8] * QSCALE; x[3] = p[9] * QSCALE;
+        }
+        uint4 f;
+        split_pair(x[0], x[1], f.x, f.y);
+        split_pair(x[2], x[3], f.z, f.w);
+        return f;
+    }
 
     __device__ __forceinline__ void init(const float *qg, int G, int lane) {
-        const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (g < G) {
-                const float *p = qg + g * D + 16 * ks + 2 * t;
-                x[0] = p[0] * QSCALE; x[1] = p[1] * QSCALE; x[2] = p[8] * QSCALE; x[3] = p[9] * QSCALE;
-            }
-            split_pair(x[0], x[1], qa[ks][0], qa[ks][1]);
-            split_pair(x[2], x[3], qa[ks][2], qa[ks][3]);
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        for (int ks = 0; ks < 16; ++ks) qa[ks] = make_qfrag(qg, G, ks, lane);
         m_run = -INFINITY;
         l_run = 0.f;
     }
 
-    template <bool MASK>
-    __device__ __forceinline__ void tile(const uint8_t *tp, int valid, int lane) {
+    // S[head g][tokens 2t, 2t+1] of tiles A (s[0], s[1]) and B (s[2], s[3]).
+    __device__ __forceinline__ void scores(const uint8_t *tA, const float *fA, int lane, float (&s)[4]) const {
+        const uint8_t *tB = tA + L::BYTES;
+        const float *fB = fA + C::SF_TILE;
         const int t = lane & 3;
-        // ---- scores S[head g][tokens 2t, 2t+1] ------------------------------
-        float s0 = 0.f, s1 = 0.f;
+        s[0] = s[1] = s[2] = s[3] = 0.f;
         if constexpr (L::KP == PART_Q4) {
-            const uint4 kw0 = lds128(tp + L::KC + lane * 16);
-            const uint4 kw1 = lds128(tp + L::KC + 512 + lane * 16);
-            const uint4 ks0 = lds128(tp + L::KS + t * 32);
-            const uint4 ks1 = lds128(tp + L::KS + t * 32 + 16);
-            const uint32_t kw[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
-            const uint32_t kd[8] = {ks0.x, ks0.y, ks0.z, ks0.w, ks1.x, ks1.y, ks1.z, ks1.w};
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t w = kw[b], w2 = kw[b] >> 8;
-                mma16816(acc, qa[2 * b], h2_as_u32(q4_lo_pair(w)), h2_as_u32(q4_hi_pair(w)));
-                mma16816(acc, qa[2 * b + 1], h2_as_u32(q4_lo_pair(w2)), h2_as_u32(q4_hi_pair(w2)));
-                const float2 d = __half22float2(u32_as_h2(kd[b]));
-                s0 = fmaf(acc[0] + acc[2], d.x, s0);
-                s1 = fmaf(acc[1] + acc[3], d.y, s1);
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 kA = lds128(tA + L::KC + hf * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + hf * 512 + lane * 16);
+                const float4 dA0 = lds128f(fA + t * C::KSTRIDE + 8 * hf), dA1 = lds128f(fA + t * C::KSTRIDE + 8 * hf + 4);
+                const float4 dB0 = lds128f(fB + t * C::KSTRIDE + 8 * hf), dB1 = lds128f(fB + t * C::KSTRIDE + 8 * hf + 4);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int b = 4 * hf + bb;
+                    const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
+                    float a[4], c[4];
+                    mma_z(a, qa[2 * b], h2_as_u32(q4_lo_pair(wA)), h2_as_u32(q4_hi_pair(wA)));
+                    mma_z(c, qa[2 * b], h2_as_u32(q4_lo_pair(wB)), h2_as_u32(q4_hi_pair(wB)));
+                    mma_acc(a, qa[2 * b + 1], h2_as_u32(q4_lo_pair(wA >> 8)), h2_as_u32(q4_hi_pair(wA >> 8)));
+                    mma_acc(c, qa[2 * b + 1], h2_as_u32(q4_lo_pair(wB >> 8)), h2_as_u32(q4_hi_pair(wB >> 8)));
+                    const float2 da = f2_at(dA0, dA1, bb), db = f2_at(dB0, dB1, bb);
+                    s[0] = fmaf(a[0] + a[2], da.x, s[0]);
+                    s[1] = fmaf(a[1] + a[3], da.y, s[1]);
+                    s[2] = fmaf(c[0] + c[2], db.x, s[2]);
+                    s[3] = fmaf(c[1] + c[3], db.y, s[3]);
+                }
             }
         } else {
-            uint4 kwv[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) kwv[c] = lds128(tp + L::KC + c * 512 + lane * 16);
-            const uint4 ks = lds128(tp + L::KS + t * 16);
-            const uint32_t kd[4] = {ks.x, ks.y, ks.z, ks.w};
+            const float4 dA0 = lds128f(fA + t * C::KSTRIDE), dA1 = lds128f(fA + t * C::KSTRIDE + 4);
+            const float4 dB0 = lds128f(fB + t * C::KSTRIDE), dB1 = lds128f(fB + t * C::KSTRIDE + 4);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t ws[4] = {kwv[q].x, kwv[q].y, kwv[q].z, kwv[q].w};
+                const uint4 kA = lds128(tA + L::KC + q * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + q * 512 + lane * 16);
+                float a[4], c[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const uint32_t wb = ws[j] ^ 0x80808080u;
-                    mma16816(acc, qa[4 * q + j], h2_as_u32(i8_pair(wb, 0x4140u)), h2_as_u32(i8_pair(wb, 0x4342u)));
+                    const uint32_t wA = u4_at(kA, j) ^ 0x80808080u, wB = u4_at(kB, j) ^ 0x80808080u;
+                    if (j == 0) {
+                        mma_z(a, qa[4 * q], h2_as_u32(i8_pair(wA, 0x4140u)), h2_as_u32(i8_pair(wA, 0x4342u)));
+                        mma_z(c, qa[4 * q], h2_as_u32(i8_pair(wB, 0x4140u)), h2_as_u32(i8_pair(wB, 0x4342u)));
+                    } else {
+                        mma_acc(a, qa[4 * q + j], h2_as_u32(i8_pair(wA, 0x4140u)), h2_as_u32(i8_pair(wA, 0x4342u)));
+                        mma_acc(c, qa[4 * q + j], h2_as_u32(i8_pair(wB, 0x4140u)), h2_as_u32(i8_pair(wB, 0x4342u)));
+                    }
                 }
-                const float2 d = __half22float2(u32_as_h2(kd[q]));
-                s0 = fmaf(acc[0] + acc[2], d.x, s0);
-                s1 = fmaf(acc[1] + acc[3], d.y, s1);
-            }
-        }
-        if (MASK) {
-            if (2 * t >= valid) s0 = -INFINITY;
-            if (2 * t + 1 >= valid) s1 = -INFINITY;
-        }
-        // ---- online softmax for head g ---------------------------------------
-        float mx = fmaxf(s0, s1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const bool grow = mx > m_run;
-        if (__any_sync(0xffffffffu, grow)) {
-            const float m_new = grow ? mx : m_run;
-            const float alpha = exp2f(m_run - m_new);     // 0 on the first tile (m_run = -inf)
-            l_run *= alpha;
-            m_run = m_new;
-            const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * t);       // head 2t
-            const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);   // head 2t+1
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                o[i][0] *= a_lo; o[i][2] *= a_lo;
-                o[i][1] *= a_hi; o[i][3] *= a_hi;
-            }
-        }
-        const float p0 = exp2f(s0 - m_run), p1 = exp2f(s1 - m_run);
-        l_run += p0 + p1;
-        // ---- values: o[dims][heads] += V^T P ------------------------------------
-        if constexpr (L::VP == PART_Q4) {
-            const uint4 vw0 = lds128(tp + L::VC + lane * 16);
-            const uint4 vw1 = lds128(tp + L::VC + 512 + lane * 16);
-            const uint4 vs0 = lds128(tp + L::VS + t * 32);
-            const uint4 vs1 = lds128(tp + L::VS + t * 32 + 16);
-            const uint32_t vw[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
-            const uint32_t vd[8] = {vs0.x, vs0.y, vs0.z, vs0.w, vs1.x, vs1.y, vs1.z, vs1.w};
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const float2 d = __half22float2(u32_as_h2(vd[b]));
-                float x0 = p0 * d.x, x1 = p1 * d.y;
-                if (MASK) {           // scales of tokens past the end may hold anything
-                    if (2 * t >= valid) x0 = 0.f;
-                    if (2 * t + 1 >= valid) x1 = 0.f;
-                }
-                uint32_t hi, lo;
-                split_pair(x0, x1, hi, lo);
-                const uint32_t w = vw[b], w2 = vw[b] >> 8;
-                const uint32_t a0 = h2_as_u32(q4_lo_pair(w)), a1 = h2_as_u32(q4_hi_pair(w));
-                const uint32_t c0 = h2_as_u32(q4_lo_pair(w2)), c1 = h2_as_u32(q4_hi_pair(w2));
-                const uint32_t A0[4] = {a0, a1, a0, a1};
-                const uint32_t A1[4] = {c0, c1, c0, c1};
-                mma16816(o[2 * b], A0, hi, lo);
-                mma16816(o[2 * b + 1], A1, hi, lo);
-            }
-        } else {
-            const uint4 vs = lds128(tp + L::VS + t * 16);
-            const uint32_t vd[4] = {vs.x, vs.y, vs.z, vs.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 vw = lds128(tp + L::VC + q * 512 + lane * 16);
-                const uint32_t ws[4] = {vw.x, vw.y, vw.z, vw.w};
-                const float2 d = __half22float2(u32_as_h2(vd[q]));
-                float x0 = p0 * d.x, x1 = p1 * d.y;
-                if (MASK) {
-                    if (2 * t >= valid) x0 = 0.f;
-                    if (2 * t + 1 >= valid) x1 = 0.f;
-                }
-                uint32_t hi, lo;
-                split_pair(x0, x1, hi, lo);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t wb = ws[j] ^ 0x80808080u;
-                    const uint32_t a0 = h2_as_u32(i8_pair(wb, 0x4140u)), a1 = h2_as_u32(i8_pair(wb, 0x4342u));
-                    const uint32_t A[4] = {a0, a1, a0, a1};
-                    mma16816(o[4 * q + j], A, hi, lo);
-                }
+                const float2 da = f2_at(dA0, dA1, q), db = f2_at(dB0, dB1, q);
+                s[0] = fmaf(a[0] + a[2], da.x, s[0]);
+                s[1] = fmaf(a[1] + a[3], da.y, s[1]);
+                s[2] = fmaf(c[0] + c[2], db.x, s[2]);
+                s[3] = fmaf(c[1] + c[3], db.y, s[3]);
             }
         }
     }
 
-    // Per-warp result into the CTA merge buffers.
-    __device__ __forceinline__ void warp_stats(int lane, float &m, float &l) {
-        float lr = l_run;
-        lr += __shfl_xor_sync(0xffffffffu, lr, 1);
-        lr += __shfl_xor_sync(0xffffffffu, lr, 2);
-        m = m_run;
-        l = lr;
+    // Scores, softmax update, and the hand-over slot: p (lane*4 .. +4) and the
+    // rescale factor of head g at [128 + g].
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tA, const float *fA, int vA, int vB, int lane, float *slot) {
+        const int g = lane >> 2, t = lane & 3;
+        float s[4];
+        scores(tA, fA, lane, s);
+        if (MASK) {
+            if (2 * t >= vA) s[0] = -INFINITY;
+            if (2 * t + 1 >= vA) s[1] = -INFINITY;
+            if (2 * t >= vB) s[2] = -INFINITY;
+            if (2 * t + 1 >= vB) s[3] = -INFINITY;
+        }
+        float mx = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);       // mx is finite: every item has a valid token
+        const float alpha = ex2(m_run - m_new);      // 1 when the max did not grow; 0 on the first item
+        l_run *= alpha;
+        m_run = m_new;
+        float p[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = ex2(s[i] - m_run);
+        l_run += (p[0] + p[1]) + (p[2] + p[3]);
+        sts128(slot + lane * 4, make_uint4(__float_as_uint(p[0]), __float_as_uint(p[1]), __float_as_uint(p[2]),
+                                           __float_as_uint(p[3])));
+        if (t == 0) slot[128 + g] = alpha;
     }
+    // An item whose page could not be read: nothing to add, nothing to rescale.
+    __device__ __forceinline__ void skip(int lane, float *slot) {
+        if (lane < 8) slot[128 + lane] = 1.f;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// PV warp: o[dims][heads] += V^T P for one work item
+// ---------------------------------------------------------------------------
+template <int FMT> struct PvWarp {
+    using L = TileLayout<FMT>;
+    float o[16][4];        // m-tile mt: o[16 mt + g (+8)][heads 2t, 2t+1]
+
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    }
+
+    // B operand of the value product for one block: P' = p * dV as an exact
+    // fp16 pair (hi, lo): hi = rn(p_hi dV), r = p_hi dV - hi (exact, from the
+    // fused multiply-add), lo = rn(p_lo dV + r).
+    __device__ __forceinline__ static void pscale(uint32_t dv2, uint32_t ph, uint32_t pl, uint32_t &hi, uint32_t &lo) {
+        const __half2 d = u32_as_h2(dv2);
+        const __half2 h = __hmul2(u32_as_h2(ph), d);
+        const __half2 r = __hfma2(u32_as_h2(ph), d, __hneg2(h));
+        hi = h2_as_u32(h);
+        lo = h2_as_u32(__hfma2(u32_as_h2(pl), d, r));
+    }
+    // Block b of both tiles: A = [V of tile A tokens 2t, 2t+1 | of tile B], k =
+    // 16 tokens; B = P' of the same tokens, once with the hi and once with the
+    // lo halves of the exact fp16 pair.
+    __device__ __forceinline__ void pv_q4(int b, uint32_t wA, uint32_t wB, uint32_t dA, uint32_t dB,
+                                          uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
+        uint32_t hA, lA, hB, lB;
+        pscale(dA, phA, plA, hA, lA);
+        pscale(dB, phB, plB, hB, lB);
+        const uint4 m0 = make_uint4(h2_as_u32(q4_lo_pair(wA)), h2_as_u32(q4_hi_pair(wA)),
+                                    h2_as_u32(q4_lo_pair(wB)), h2_as_u32(q4_hi_pair(wB)));
+        const uint4 m1 = make_uint4(h2_as_u32(q4_lo_pair(wA >> 8)), h2_as_u32(q4_hi_pair(wA >> 8)),
+                                    h2_as_u32(q4_lo_pair(wB >> 8)), h2_as_u32(q4_hi_pair(wB >> 8)));
+        mma_acc(o[2 * b], m0, hA, hB);
+        mma_acc(o[2 * b + 1], m1, hA, hB);
+        mma_acc(o[2 * b], m0, lA, lB);
+        mma_acc(o[2 * b + 1], m1, lA, lB);
+    }
+    __device__ __forceinline__ void pv_i8(int q, const uint4 &wvA, const uint4 &wvB, uint32_t dA, uint32_t dB,
+                                          uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
+        uint32_t hA, lA, hB, lB;
+        pscale(dA, phA, plA, hA, lA);
+        pscale(dB, phB, plB, hB, lB);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t xa = u4_at(wvA, j) ^ 0x80808080u, xb = u4_at(wvB, j) ^ 0x80808080u;
+            const uint4 m = make_uint4(h2_as_u32(i8_pair(xa, 0x4140u)), h2_as_u32(i8_pair(xa, 0x4342u)),
+                                       h2_as_u32(i8_pair(xb, 0x4140u)), h2_as_u32(i8_pair(xb, 0x4342u)));
+            mma_acc(o[4 * q + j], m, hA, hB);
+            mma_acc(o[4 * q + j], m, lA, lB);
+        }
+    }
+
+    // Rescale (factors of heads 2t, 2t+1 from the slot) and accumulate the item.
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tA, int vA, int vB, bool ok, int lane, const float4 &p,
+                                         float2 al) {
+        const int t = lane & 3;
+        if (__any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                o[i][0] *= al.x; o[i][2] *= al.x;
+                o[i][1] *= al.y; o[i][3] *= al.y;
+            }
+        }
+        if (!ok) return;
+        const uint8_t *tB = tA + L::BYTES;
+        uint32_t phA, plA, phB, plB;     // p of tokens 2t, 2t+1 as fp16 hi + lo pairs
+        split_pair(p.x, p.y, phA, plA);
+        split_pair(p.z, p.w, phB, plB);
+        // zero the scales of tokens past the end (their bytes may hold anything)
+        const uint32_t mA = MASK ? ((2 * t < vA ? 0xFFFFu : 0u) | (2 * t + 1 < vA ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
+        const uint32_t mB = MASK ? ((2 * t < vB ? 0xFFFFu : 0u) | (2 * t + 1 < vB ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
+        if constexpr (L::VP == PART_Q4) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 wvA = lds128(tA + L::VC + hf * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + hf * 512 + lane * 16);
+                const uint4 eA = lds128(tA + L::VS + t * 32 + hf * 16);   // (dV[2t][b], dV[2t+1][b]), b = 4 hf + bb
+                const uint4 eB = lds128(tB + L::VS + t * 32 + hf * 16);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    pv_q4(4 * hf + bb, u4_at(wvA, bb), u4_at(wvB, bb), u4_at(eA, bb) & mA, u4_at(eB, bb) & mB, phA,
+                          plA, phB, plB);
+            }
+        } else {
+            const uint4 eA = lds128(tA + L::VS + t * 16);                 // (dV[2t][q], dV[2t+1][q]), q = 0..3
+            const uint4 eB = lds128(tB + L::VS + t * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 wvA = lds128(tA + L::VC + q * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + q * 512 + lane * 16);
+                pv_i8(q, wvA, wvB, u4_at(eA, q) & mA, u4_at(eB, q) & mB, phA, plA, phB, plB);
+            }
+        }
+    }
+
     // Add this warp's o (scaled per head) into o_s[8][256].
     __device__ __forceinline__ void accumulate(float *o_s, const float *scale, int lane) {
         const int g = lane >> 2, t = lane & 3;
@@ -236,8 +387,6 @@ template <int FMT> struct MmaCompute {
             atomicAdd(o_s + (2 * t + 1) * D + d0 + 8, o[mt][3] * sc1);
         }
     }
-    // head whose (m, l) this lane reports; -1 if none
-    __device__ __forceinline__ int stats_head(int lane) { return (lane & 3) == 0 ? (lane >> 2) : -1; }
 };
 
 // ---------------------------------------------------------------------------
@@ -247,6 +396,7 @@ template <int FMT> struct MmaCompute {
 // ---------------------------------------------------------------------------
 template <int FMT, int GT> struct AluCompute {
     using L = TileLayout<FMT>;
+    static constexpr int TPI = 1;
     float qr[GT][8];
     float o[GT][8];
     float m_run[2], l_run[2];   // heads 2(l%4), 2(l%4)+1
@@ -417,18 +567,24 @@ template <int FMT, int GT> struct AluCompute {
         }
     }
 
-    __device__ __forceinline__ void warp_stats(int lane, float &m, float &l) {
-        // lanes 0..3 report heads 2l, 2l+1 via the caller; reduce l over tokens
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tp, const float *, int vA, int, int lane) {
+        tile<MASK>(tp, vA, lane);
+    }
+
+    __device__ __forceinline__ void report(int lane, float *m_s, float *l_s) {
         float l0 = l_run[0], l1 = l_run[1];
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, off);
             l1 += __shfl_xor_sync(0xffffffffu, l1, off);
         }
-        l_run[0] = l0;
-        l_run[1] = l1;
-        m = m_run[0];
-        l = l0;
+        if (lane < 4) {
+            m_s[2 * lane] = m_run[0];
+            m_s[2 * lane + 1] = m_run[1];
+            l_s[2 * lane] = l0;
+            l_s[2 * lane + 1] = l1;
+        }
     }
     __device__ __forceinline__ void accumulate(float *o_s, const float *scale, int lane) {
 #pragma unroll
@@ -439,183 +595,535 @@ template <int FMT, int GT> struct AluCompute {
 };
 
 // ---------------------------------------------------------------------------
-// Kernel scaffold
+// Merge of one (sequence, KV head) group: units [u0, u1) of the workspace ->
+// the G output rows starting at out_row.  M = max m_u, L = sum l_u 2^(m_u - M),
+// o = sum 2^(m_u - M) o_u / L, then H/16 if V was stored rotated.  Runs on the
+// first NTH threads of the CTA (named barrier bar_id); sm: COMBINE_SMEM floats.
+// All (m, l) pairs are staged in shared memory first, so the loads of the
+// partial outputs are independent of each other and issue back to back.
 // ---------------------------------------------------------------------------
-template <int FMT, bool TC, int GT>
-__global__ void __launch_bounds__(NTHREADS, 1)
-decode_kernel(const uint8_t *__restrict__ pool, PoolGeom geo, int layer, const float *__restrict__ q,
-              const int32_t *__restrict__ page_table, int max_pages, const int32_t *__restrict__ plan, int n_q_heads,
-              int G, float *__restrict__ ws, int32_t *status) {
+template <int NTH>
+__device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t out_row, int inverse_fwht,
+                              uint16_t *out_bf16, float *out_f32, float *sm, int bar_id) {
+    constexpr int NWARP = NTH / 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int stride = ws_unit_floats(G);
+    float *o_s = sm;                              // [8][256] accumulated outputs
+    float *f_s = sm + 8 * D;                      // [units][8] weights 2^(m_u - M)
+    float *l_s = f_s + 8 * COMBINE_MAX_UNITS;     // [units][8] sums l_u
+    float *Ms = l_s + 8 * COMBINE_MAX_UNITS;      // [8]
+    float *Ls = Ms + 8;                           // [8]
+    for (int i = tid; i < 8 * D; i += NTH) o_s[i] = 0.f;
+    if (tid < 8) {
+        Ms[tid] = -INFINITY;
+        Ls[tid] = 0.f;
+    }
+    for (int c0 = u0; c0 < u1; c0 += COMBINE_MAX_UNITS) {     // chunks of units (one pass in practice)
+        const int n = min(COMBINE_MAX_UNITS, u1 - c0);
+        // stage m and l of every (unit, head)
+        for (int i = tid; i < n * 8; i += NTH) {
+            const int uu = i >> 3, h = i & 7;
+            const float *p = ws + (size_t)(c0 + uu) * stride + G * D;
+            f_s[i] = h < G ? __ldcg(p + h) : -INFINITY;
+            l_s[i] = h < G ? __ldcg(p + 8 + h) : 0.f;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+        // new running max per head; rescale what is accumulated so far
+        if (tid < 8) {
+            float M = Ms[tid];
+            for (int uu = 0; uu < n; ++uu) M = fmaxf(M, f_s[uu * 8 + tid]);
+            const float scale_old = Ms[tid] == -INFINITY ? 0.f : exp2f(Ms[tid] - M);
+            float L = Ls[tid] * scale_old;
+            for (int uu = 0; uu < n; ++uu) {
+                const float m = f_s[uu * 8 + tid];
+                const float f = m == -INFINITY ? 0.f : exp2f(m - M);
+                f_s[uu * 8 + tid] = f;
+                L = fmaf(l_s[uu * 8 + tid], f, L);
+            }
+            l_s[tid] = scale_old;            // reuse: factor for the accumulators of this head
+            Ms[tid] = M;
+            Ls[tid] = L;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+        // rescale earlier chunks (only with more than COMBINE_MAX_UNITS units)
+        if (c0 > u0 && warp == 0)
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o_s[h * D + lane * 8 + i] *= l_s[h];
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+        // warps per head: warp w takes head w % G and every wph-th unit; the unit
+        // loads are independent of each other (weights come from shared memory)
+        const int wph = NWARP >= G ? NWARP / G : 1;
+        if (warp < wph * G) {
+            const int h = warp % G, part = warp / G;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int uu = part; uu < n; uu += wph) {
+                const float f = f_s[uu * 8 + h];
+                const float *p = ws + (size_t)(c0 + uu) * stride + h * D + lane * 8;
+                const float4 a = __ldcg(reinterpret_cast<const float4 *>(p));
+                const float4 b = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
+                acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+                acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
+                acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
+                acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) atomicAdd(o_s + h * D + lane * 8 + i, acc[i]);
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+    }
+    // warp h finishes head h
+    for (int h = warp; h < G; h += NWARP) {
+        float x[8];
+        const float inv = 1.0f / Ls[h];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = o_s[h * D + lane * 8 + i] * inv;
+        if (inverse_fwht) {
+#pragma unroll
+            for (int hh = 1; hh < 8; hh <<= 1)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if ((i & hh) == 0) {
+                        const float a = x[i], b = x[i + hh];
+                        x[i] = a + b;
+                        x[i + hh] = a - b;
+                    }
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const bool upper = (lane & m) != 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float other = __shfl_xor_sync(0xffffffffu, x[i], m);
+                    x[i] = upper ? other - x[i] : x[i] + other;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] *= 0.0625f;
+        }
+        const size_t off = (size_t)(out_row + h) * D + lane * 8;
+        if (out_f32) {
+            float4 *o = reinterpret_cast<float4 *>(out_f32 + off);
+            o[0] = make_float4(x[0], x[1], x[2], x[3]);
+            o[1] = make_float4(x[4], x[5], x[6], x[7]);
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+            pk[i] = *reinterpret_cast<const uint32_t *>(&v);
+        }
+        *reinterpret_cast<uint4 *>(out_bf16 + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
+struct DecodeArgs {
+    const uint8_t *pool;
+    PoolGeom geo;
+    int layer;
+    const float *q;
+    const int32_t *page_table;
+    int max_pages;
+    const int32_t *plan;
+    int n_q_heads;
+    int G;
+    float *ws;
+    int32_t *status;
+    int inverse_fwht;      // fused combine: un-rotate the output
+    uint16_t *out_bf16;    // fused combine outputs (NULL: write partials only)
+    float *out_f32;
+};
+
+// ---------------------------------------------------------------------------
+// Shared pieces of both kernels
+// ---------------------------------------------------------------------------
+// Plan entry check; on failure write an empty partial so that the merge ignores
+// the unit.
+__device__ __forceinline__ bool unit_ok(const DecodeArgs &A, int seq, int kvh, int t0, int t1, float *wsu) {
+    const bool ok = A.plan[0] == PLAN_MAGIC && seq >= 0 && seq < A.plan[2] && kvh >= 0 &&
+                    kvh < A.geo.n_kv_heads && t0 >= 0 && t0 < t1 && (t0 % STEP_TOKENS) == 0 &&
+                    t1 <= A.max_pages * PAGE;
+    if (!ok) {
+        if (threadIdx.x == 0) status_or(A.status, KVQ_STATUS_BAD_PLAN);
+        for (int i = threadIdx.x; i < A.G * D; i += blockDim.x) wsu[i] = 0.f;
+        if (threadIdx.x < 8) {
+            wsu[A.G * D + threadIdx.x] = -INFINITY;
+            wsu[A.G * D + 8 + threadIdx.x] = 0.f;
+        }
+    }
+    return ok;
+}
+
+// Copy warp: stream the unit's 64-token steps into the stage ring.  All 32
+// lanes fetch the page slots of 32 pages at a time (one load round trip per 32
+// pages instead of one per step); lane 0 waits for free stages and issues the
+// bulk copies.
+template <int NS, int STAGE_BYTES, int TILE_BYTES>
+__device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                          int *stage_ok, int seq, int kvh, int t0, int n_steps, int lane) {
+    const uint8_t *head_base = A.pool + (int64_t)A.layer * A.geo.layer_stride + (int64_t)kvh * A.geo.page_bytes;
+    const int32_t *pt = A.page_table + (int64_t)seq * A.max_pages;
+    const uint64_t pol = policy_evict_first();
+    const int page0 = t0 >> 8;
+    int chunk = -1, my_slot = -1;
+    bool stop = false;
+    for (int i = 0; i < n_steps; ++i) {
+        const int tok = t0 + i * STEP_TOKENS;
+        const int rel = (tok >> 8) - page0;
+        if ((rel >> 5) != chunk) {
+            chunk = rel >> 5;
+            const int pg = page0 + 32 * chunk + lane;
+            my_slot = pg < A.max_pages ? __ldg(pt + pg) : -1;
+        }
+        const int slot = __shfl_sync(0xffffffffu, my_slot, rel & 31);
+        if (lane == 0 && !stop) {
+            const int si = i % NS;
+            if (i >= NS && !mbar_wait_bounded(&empty[si], ((i / NS) - 1) & 1, WAIT_LIMIT_NS)) {
+                status_or(A.status, KVQ_STATUS_TIMEOUT);
+                stop = true;
+            } else if (slot < 0 || slot >= A.geo.n_pages) {
+                status_or(A.status, KVQ_STATUS_BAD_SLOT);
+                stage_ok[si] = 0;
+                mbar_arrive(&full[si]);
+            } else {
+                stage_ok[si] = 1;
+                const uint8_t *src = head_base + (int64_t)slot * A.geo.slot_stride + ((tok & 255) >> 3) * TILE_BYTES;
+                mbar_arrive_expect_tx(&full[si], STAGE_BYTES);
+                bulk_g2s(smem + si * STAGE_BYTES, src, STAGE_BYTES, &full[si], pol);
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// After the warps' states are in m_s/l_s [n_rep][8] and o_s [8][256] (scaled to
+// M_s): write the unit's partial; with FUSED, the last CTA of the (sequence, KV
+// head) group merges the group.  Runs on the NCT merge threads (bar 1).
+template <bool FUSED, int NCT>
+__device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_s, const float *m_s, const float *l_s,
+                                            const float *M_s, int n_rep, float *wsu, int seq, int kvh, int n_units,
+                                            int *s_last, uint8_t *smem) {
+    const int G = A.G;
+    for (int i = threadIdx.x; i < G * D; i += NCT) wsu[i] = o_s[i];
+    if (threadIdx.x < 8) {
+        const int h = threadIdx.x;
+        float Lh = 0.f;
+        for (int w = 0; w < n_rep; ++w) {
+            const float mw = m_s[w * 8 + h];
+            if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M_s[h]);
+        }
+        wsu[G * D + h] = M_s[h];
+        wsu[G * D + 8 + h] = Lh;
+    }
+    if constexpr (FUSED) {
+        const int32_t *start = A.plan + PLAN_HEADER + 4 * n_units;
+        const int grp = seq * A.geo.n_kv_heads + kvh;
+        int *counter = reinterpret_cast<int *>(A.ws + (size_t)n_units * ws_unit_floats(G)) + grp;
+        __threadfence();
+        asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+        if (threadIdx.x == 0) {
+            const int n_grp = start[grp + 1] - start[grp];
+            const int old = atomicAdd(counter, 1);
+            *s_last = old == n_grp - 1;
+            if (*s_last) *counter = 0;         // every unit of the group has arrived: reset for the next launch
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+        if (*s_last) {
+            __threadfence();
+            combine_group<NCT>(A.ws, G, start[grp], start[grp + 1], (int64_t)seq * A.n_q_heads + (int64_t)kvh * G,
+                               A.inverse_fwht, A.out_bf16, A.out_f32, reinterpret_cast<float *>(smem), 1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core kernel
+// ---------------------------------------------------------------------------
+template <int FMT, bool FUSED>
+__global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(const DecodeArgs A) {
     using L = TileLayout<FMT>;
-    using S = Smem<FMT>;
+    using C = TcCfg<FMT>;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::BAR_OFF);
-    uint64_t *empty = full + S::NS;
-    int *stage_ok = reinterpret_cast<int *>(empty + S::NS);
-    __shared__ int s_abort;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *ready = full + C::NS;            // fp32 K scales of the stage are written
+    uint64_t *empty = ready + C::NS;           // every item of the stage is done
+    uint64_t *p_full = empty + C::NS;          // QK -> PV slot written
+    uint64_t *p_empty = p_full + C::NQK * C::DP;
+    int *stage_ok = reinterpret_cast<int *>(p_empty + C::NQK * C::DP);
+    __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.x;
-    const int32_t *U = plan + PLAN_HEADER + 4 * u;
+    const int32_t *U = A.plan + PLAN_HEADER + 4 * u;
     const int seq = U[0], kvh = U[1], t0 = U[2], t1 = U[3];
-    float *wsu = ws + (size_t)u * ws_unit_floats(G);
-
-    const bool plan_ok = plan[0] == PLAN_MAGIC && seq >= 0 && seq < plan[2] && kvh >= 0 && kvh < geo.n_kv_heads &&
-                         t0 >= 0 && t0 < t1 && (t0 % STEP_TOKENS) == 0 && t1 <= max_pages * PAGE;
-    if (!plan_ok) {   // write an empty partial so that the merge ignores this unit
-        if (threadIdx.x == 0) status_or(status, KVQ_STATUS_BAD_PLAN);
-        for (int i = threadIdx.x; i < G * D; i += blockDim.x) wsu[i] = 0.f;
-        if (threadIdx.x < 8) {
-            wsu[G * D + threadIdx.x] = -INFINITY;
-            wsu[G * D + 8 + threadIdx.x] = 0.f;
-        }
-        return;
-    }
+    const int G = A.G;
+    const int n_units = A.plan[1];
+    float *wsu = A.ws + (size_t)u * ws_unit_floats(G);
+    if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;
     const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
+    const int n_items = (t1 - t0 + 2 * TILE - 1) / (2 * TILE);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S::NS; ++i) {
+        for (int i = 0; i < C::NS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], NW);
+            mbar_init(&ready[i], 32);                    // every lane of the scale warp arrives
+            mbar_init(&empty[i], 32 * C::ITEMS_PER_STAGE);
         }
-        s_abort = 0;
+        for (int i = 0; i < C::NQK * C::DP; ++i) {      // every lane of the QK / PV warp arrives
+            mbar_init(&p_full[i], 32);
+            mbar_init(&p_empty[i], 32);
+        }
         fence_mbar_init();
     }
     __syncthreads();
 
-    const uint8_t *head_base = pool + (int64_t)layer * geo.layer_stride + (int64_t)kvh * geo.page_bytes;
-    const int32_t *pt = page_table + (int64_t)seq * max_pages;
-
-    if (warp == NW) {
-        // ------------------------------ producer --------------------------------
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            for (int i = 0; i < n_steps; ++i) {
-                const int si = i % S::NS;
-                if (i >= S::NS) {
-                    if (!mbar_wait_bounded(&empty[si], ((i / S::NS) - 1) & 1, WAIT_LIMIT_NS)) {
-                        status_or(status, KVQ_STATUS_TIMEOUT);
-                        atomicExch(&s_abort, 1);
-                        break;
-                    }
-                }
-                const int tok = t0 + i * STEP_TOKENS;
-                const int slot = pt[tok >> 8];
-                if (slot < 0 || slot >= geo.n_pages) {
-                    status_or(status, KVQ_STATUS_BAD_SLOT);
-                    stage_ok[si] = 0;
-                    mbar_arrive(&full[si]);
-                    continue;
-                }
-                stage_ok[si] = 1;
-                const uint8_t *src = head_base + (int64_t)slot * geo.slot_stride + ((tok & 255) >> 3) * L::BYTES;
-                mbar_arrive_expect_tx(&full[si], S::STAGE_BYTES);
-                bulk_g2s(smem + si * S::STAGE_BYTES, src, S::STAGE_BYTES, &full[si], pol);
-            }
-        }
-    } else {
-        // ------------------------------ consumers -------------------------------
-        float *pbuf = reinterpret_cast<float *>(smem + S::BAR_OFF + S::NS * 16 + S::NS * 4 + 16);  // unused by MMA
-        (void)pbuf;
-        const float *qg = q + ((int64_t)seq * n_q_heads + (int64_t)kvh * G) * D;
-        __shared__ float p_bufs[TC ? 1 : NW * 64];
-        typename std::conditional<TC, MmaCompute<FMT>, AluCompute<FMT, GT>>::type C;
-        if constexpr (TC) C.init(qg, G, lane);
-        else C.init(qg, G, lane, p_bufs + warp * 64);
-
+    if (warp == C::COPY_WARP) {
+        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
+        return;
+    }
+    if (warp == C::SCALE_WARP) {
         for (int i = 0; i < n_steps; ++i) {
-            const int si = i % S::NS;
-            if (!mbar_wait_bounded(&full[si], (i / S::NS) & 1, WAIT_LIMIT_NS)) {
-                if (lane == 0) { status_or(status, KVQ_STATUS_TIMEOUT); atomicExch(&s_abort, 1); }
+            const int si = i % C::NS;
+            if (!mbar_wait_bounded(&full[si], (i / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
-            const int tile_tok = t0 + i * STEP_TOKENS + warp * TILE;
-            const int valid = t1 - tile_tok;
-            if (stage_ok[si] && valid > 0) {
-                const uint8_t *tp = smem + si * S::STAGE_BYTES + warp * L::BYTES;
-                if (valid >= TILE) C.template tile<false>(tp, TILE, lane);
-                else C.template tile<true>(tp, valid, lane);
-            }
+            if (stage_ok[si])
+                convert_stage_scales<FMT>(smem + si * C::STAGE_BYTES,
+                                          reinterpret_cast<float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES), lane);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[si]);
+            mbar_arrive(&ready[si]);
         }
+        return;
+    }
 
-        // ------------------------------ CTA merge -------------------------------
-        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));           // all consumers done with the ring
-        float *o_s = reinterpret_cast<float *>(smem);             // [8][256]
-        float *m_s = o_s + 8 * D;                                 // [NW][8]
-        float *l_s = m_s + NW * 8;                                // [NW][8]
-        float *M_s = l_s + NW * 8;                                // [8]
-        float *sc_s = M_s + 8;                                    // [8] (unused slot)
-        (void)sc_s;
-        for (int i = threadIdx.x; i < 8 * D; i += NW * 32) o_s[i] = 0.f;
-        {
-            float m, l;
-            C.warp_stats(lane, m, l);
-            if constexpr (TC) {
-                const int h = C.stats_head(lane);
-                if (h >= 0) { m_s[warp * 8 + h] = m; l_s[warp * 8 + h] = l; }
-            } else {
-                if (lane < 4) {
-                    m_s[warp * 8 + 2 * lane] = C.m_run[0];
-                    m_s[warp * 8 + 2 * lane + 1] = C.m_run[1];
-                    l_s[warp * 8 + 2 * lane] = C.l_run[0];
-                    l_s[warp * 8 + 2 * lane + 1] = C.l_run[1];
-                }
+    float *pring = reinterpret_cast<float *>(smem + C::POFF);
+    constexpr int NCT = 2 * C::NQK * 32;       // merge threads: QK + PV warps
+    const bool is_qk = warp < C::NQK;
+    const int pw = is_qk ? warp : warp - C::NQK;    // pair index
+    QkWarp<FMT> qk;
+    PvWarp<FMT> pv;
+    if (is_qk) {
+        qk.init(A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D, G, lane);
+        int k = 0;
+        for (int it = pw; it < n_items; it += C::NQK, ++k) {
+            const int st = (2 * it) >> 3, si = st % C::NS, slot = k % C::DP;
+            float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
+            if (!mbar_wait_bounded(&full[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
+                !mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
+                (k >= C::DP && !mbar_wait_bounded(&p_empty[pw * C::DP + slot], ((k / C::DP) - 1) & 1, WAIT_LIMIT_NS))) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
             }
+            const int tok = t0 + 2 * it * TILE;
+            const int vA = min(TILE, t1 - tok), vB = max(0, min(TILE, t1 - tok - TILE));
+            if (stage_ok[si]) {
+                const uint8_t *tp = smem + si * C::STAGE_BYTES + ((2 * it) & 7) * L::BYTES;
+                const float *fp = reinterpret_cast<const float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES) +
+                                  ((2 * it) & 7) * C::SF_TILE;
+                if (vA == TILE && vB == TILE) qk.template item<false>(tp, fp, vA, vB, lane, ps);
+                else qk.template item<true>(tp, fp, vA, vB, lane, ps);
+            } else {
+                qk.skip(lane, ps);
+            }
+            mbar_arrive(&p_full[pw * C::DP + slot]);
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));
-        if (threadIdx.x < 8) {
-            float M = -INFINITY;
-            for (int w = 0; w < NW; ++w) M = fmaxf(M, m_s[w * 8 + threadIdx.x]);
-            M_s[threadIdx.x] = M;
+    } else {
+        pv.init();
+        int k = 0;
+        for (int it = pw; it < n_items; it += C::NQK, ++k) {
+            const int st = (2 * it) >> 3, si = st % C::NS, slot = k % C::DP;
+            const float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
+            if (!mbar_wait_bounded(&p_full[pw * C::DP + slot], (k / C::DP) & 1, WAIT_LIMIT_NS) ||
+                !mbar_wait_bounded(&full[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            const float4 p = lds128f(ps + lane * 4);
+            const float2 al = make_float2(ps[128 + 2 * (lane & 3)], ps[128 + 2 * (lane & 3) + 1]);
+            mbar_arrive(&p_empty[pw * C::DP + slot]);
+            const int tok = t0 + 2 * it * TILE;
+            const int vA = min(TILE, t1 - tok), vB = max(0, min(TILE, t1 - tok - TILE));
+            const uint8_t *tp = smem + si * C::STAGE_BYTES + ((2 * it) & 7) * L::BYTES;
+            const bool ok = stage_ok[si] != 0;
+            if (vA == TILE && vB == TILE) pv.template item<false>(tp, vA, vB, ok, lane, p, al);
+            else pv.template item<true>(tp, vA, vB, ok, lane, p, al);
+            mbar_arrive(&empty[si]);
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));
+    }
+
+    // ---- CTA merge: QK warps report (m, l), PV warps add o ---------------------
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));               // every consumer is done with the ring
+    float *o_s = reinterpret_cast<float *>(smem);             // [8][256]
+    float *m_s = o_s + 8 * D;                                 // [NQK][8]
+    float *l_s = m_s + C::NQK * 8;                            // [NQK][8]
+    float *M_s = l_s + C::NQK * 8;                            // [8]
+    for (int i = threadIdx.x; i < 8 * D; i += NCT) o_s[i] = 0.f;
+    if (is_qk) {
+        float lr = qk.l_run;
+        lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+        lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+        if ((lane & 3) == 0) {
+            m_s[pw * 8 + (lane >> 2)] = qk.m_run;
+            l_s[pw * 8 + (lane >> 2)] = lr;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    if (threadIdx.x < 8) {
+        float M = -INFINITY;
+        for (int w = 0; w < C::NQK; ++w) M = fmaxf(M, m_s[w * 8 + threadIdx.x]);
+        M_s[threadIdx.x] = M;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    if (!is_qk) {
         float scale[8];
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
-            const float mw = m_s[warp * 8 + h];
+            const float mw = m_s[pw * 8 + h];
             scale[h] = mw == -INFINITY ? 0.f : exp2f(mw - M_s[h]);
         }
-        C.accumulate(o_s, scale, lane);
-        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32));
-        // partial: o[G][256], m[8], l[8]
-        for (int i = threadIdx.x; i < G * D; i += NW * 32) wsu[i] = o_s[i];
-        if (threadIdx.x < 8) {
-            const int h = threadIdx.x;
-            float Lh = 0.f;
-            for (int w = 0; w < NW; ++w) {
-                const float mw = m_s[w * 8 + h];
-                if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M_s[h]);
-            }
-            wsu[G * D + h] = M_s[h];
-            wsu[G * D + 8 + h] = Lh;
-        }
+        pv.accumulate(o_s, scale, lane);
     }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    finish_unit<FUSED, NCT>(A, o_s, m_s, l_s, M_s, C::NQK, wsu, seq, kvh, n_units, &s_last, smem);
 }
 
-template <int FMT, bool TC, int GT>
-cudaError_t launch_one(const uint8_t *pool, const PoolGeom &geo, int layer, const float *q, const int32_t *pt,
-                       int max_pages, const int32_t *plan, const kvq_plan_info &info, float *ws, int32_t *status,
-                       cudaStream_t s) {
-    constexpr int SMEM = Smem<FMT>::TOTAL;
-    auto k = decode_kernel<FMT, TC, GT>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return e;
-    k<<<info.n_units, NTHREADS, SMEM, s>>>(pool, geo, layer, q, pt, max_pages, plan,
-                                           info.n_kv_heads * info.group, info.group, ws, status);
+// ---------------------------------------------------------------------------
+// CUDA-core kernel (control): 8 consumer warps, one tile per item, + copy warp
+// ---------------------------------------------------------------------------
+template <int FMT> struct AluCfg {
+    static constexpr int NCW = 8;
+    static constexpr int NTHREADS = (NCW + 1) * 32;
+    static constexpr int STAGE_BYTES = 8 * TileLayout<FMT>::BYTES;
+    static constexpr int NS = FMT == KVQ_Q4_0 ? 5 : (FMT == KVQ_INT8 ? 3 : 4);
+    static constexpr int RING = NS * STAGE_BYTES;
+    static constexpr int MERGE = (COMBINE_SMEM > 8 * D + 2 * NCW * 8 + 16 ? COMBINE_SMEM : 8 * D + 2 * NCW * 8 + 16) * 4;
+    static constexpr int DATA = RING > MERGE ? RING : MERGE;
+    static constexpr int BAR_OFF = (DATA + 127) & ~127;
+    static constexpr int TOTAL = BAR_OFF + 2 * NS * 8 + NS * 4 + 16;
+};
+
+template <int FMT, int GT, bool FUSED>
+__global__ void __launch_bounds__(AluCfg<FMT>::NTHREADS, 1) decode_alu_kernel(const DecodeArgs A) {
+    using L = TileLayout<FMT>;
+    using C = AluCfg<FMT>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    int *stage_ok = reinterpret_cast<int *>(empty + C::NS);
+    __shared__ int s_last;
+    __shared__ float p_bufs[C::NCW * 64];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.x;
+    const int32_t *U = A.plan + PLAN_HEADER + 4 * u;
+    const int seq = U[0], kvh = U[1], t0 = U[2], t1 = U[3];
+    const int G = A.G;
+    const int n_units = A.plan[1];
+    float *wsu = A.ws + (size_t)u * ws_unit_floats(G);
+    if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;
+    const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
+    const int n_tiles = (t1 - t0 + TILE - 1) / TILE;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 8);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == C::NCW) {
+        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
+        return;
+    }
+    AluCompute<FMT, GT> comp;
+    comp.init(A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D, G, lane, p_bufs + warp * 64);
+    for (int it = warp; it < n_tiles; it += C::NCW) {
+        const int st = it >> 3, si = st % C::NS;
+        if (!mbar_wait_bounded(&full[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
+            if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+            break;
+        }
+        const int valid = min(TILE, t1 - (t0 + it * TILE));
+        if (stage_ok[si]) {
+            const uint8_t *tp = smem + si * C::STAGE_BYTES + (it & 7) * L::BYTES;
+            if (valid == TILE) comp.template item<false>(tp, nullptr, valid, 0, lane);
+            else comp.template item<true>(tp, nullptr, valid, 0, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[si]);
+    }
+    constexpr int NCT = C::NCW * 32;
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    float *o_s = reinterpret_cast<float *>(smem);
+    float *m_s = o_s + 8 * D;
+    float *l_s = m_s + C::NCW * 8;
+    float *M_s = l_s + C::NCW * 8;
+    for (int i = threadIdx.x; i < 8 * D; i += NCT) o_s[i] = 0.f;
+    comp.report(lane, m_s + warp * 8, l_s + warp * 8);
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    if (threadIdx.x < 8) {
+        float M = -INFINITY;
+        for (int w = 0; w < C::NCW; ++w) M = fmaxf(M, m_s[w * 8 + threadIdx.x]);
+        M_s[threadIdx.x] = M;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    float scale[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+        const float mw = m_s[warp * 8 + h];
+        scale[h] = mw == -INFINITY ? 0.f : exp2f(mw - M_s[h]);
+    }
+    comp.accumulate(o_s, scale, lane);
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    finish_unit<FUSED, NCT>(A, o_s, m_s, l_s, M_s, C::NCW, wsu, seq, kvh, n_units, &s_last, smem);
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ plan,
+                                                      int n_kv, int G, int inverse_fwht, uint16_t *out_bf16,
+                                                      float *out_f32) {
+    __shared__ float sm[COMBINE_SMEM];
+    const int grp = blockIdx.x;
+    const int seq = grp / n_kv, kvh = grp - seq * n_kv;
+    const int n_units = plan[1];
+    const int32_t *start = plan + PLAN_HEADER + 4 * n_units;
+    combine_group<256>(ws, G, start[grp], start[grp + 1], (int64_t)seq * n_kv * G + (int64_t)kvh * G, inverse_fwht,
+                       out_bf16, out_f32, sm, 1);
+}
+
+template <typename K>
+cudaError_t launch_k(K kernel, int smem_bytes, int threads, const DecodeArgs &a, int n_units, cudaStream_t s,
+                     bool &configured) {
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    kernel<<<n_units, threads, smem_bytes, s>>>(a);
     return cudaGetLastError();
 }
 
-template <int FMT>
-cudaError_t launch_fmt(bool tc, const uint8_t *pool, const PoolGeom &geo, int layer, const float *q,
-                       const int32_t *pt, int max_pages, const int32_t *plan, const kvq_plan_info &info, float *ws,
-                       int32_t *status, cudaStream_t s) {
-    if (tc) return launch_one<FMT, true, 8>(pool, geo, layer, q, pt, max_pages, plan, info, ws, status, s);
-    switch (info.group) {
-    case 4: return launch_one<FMT, false, 4>(pool, geo, layer, q, pt, max_pages, plan, info, ws, status, s);
-    case 6: return launch_one<FMT, false, 6>(pool, geo, layer, q, pt, max_pages, plan, info, ws, status, s);
-    default: return launch_one<FMT, false, 8>(pool, geo, layer, q, pt, max_pages, plan, info, ws, status, s);
+template <int FMT, bool FUSED>
+cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s) {
+    if (tc) {
+        static bool cfg = false;
+        return launch_k(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS, a, n_units, s, cfg);
+    }
+    static bool c4 = false, c6 = false, c8 = false;
+    switch (a.G) {
+    case 4: return launch_k(decode_alu_kernel<FMT, 4, FUSED>, AluCfg<FMT>::TOTAL, AluCfg<FMT>::NTHREADS, a, n_units, s, c4);
+    case 6: return launch_k(decode_alu_kernel<FMT, 6, FUSED>, AluCfg<FMT>::TOTAL, AluCfg<FMT>::NTHREADS, a, n_units, s, c6);
+    default: return launch_k(decode_alu_kernel<FMT, 8, FUSED>, AluCfg<FMT>::TOTAL, AluCfg<FMT>::NTHREADS, a, n_units, s, c8);
+    }
+}
+
+template <bool FUSED>
+cudaError_t launch_fused(int fmt, bool tc, const DecodeArgs &a, int n_units, cudaStream_t s) {
+    switch (fmt) {
+    case KVQ_INT8: return launch_fmt<KVQ_INT8, FUSED>(tc, a, n_units, s);
+    case KVQ_Q4_0: return launch_fmt<KVQ_Q4_0, FUSED>(tc, a, n_units, s);
+    default: return launch_fmt<KVQ_K8V4, FUSED>(tc, a, n_units, s);
     }
 }
 
@@ -623,15 +1131,20 @@ cudaError_t launch_fmt(bool tc, const uint8_t *pool, const PoolGeom &geo, int la
 
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
-                          const kvq_plan_info &info, float *ws, int32_t *status, cudaStream_t s) {
-    switch (fmt) {
-    case KVQ_INT8:
-        return launch_fmt<KVQ_INT8>(tensor_cores, pool, geo, layer, q, page_table, max_pages, plan, info, ws, status, s);
-    case KVQ_Q4_0:
-        return launch_fmt<KVQ_Q4_0>(tensor_cores, pool, geo, layer, q, page_table, max_pages, plan, info, ws, status, s);
-    default:
-        return launch_fmt<KVQ_K8V4>(tensor_cores, pool, geo, layer, q, page_table, max_pages, plan, info, ws, status, s);
-    }
+                          const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht, uint16_t *out_bf16,
+                          float *out_f32, cudaStream_t s) {
+    DecodeArgs a{pool, geo, layer, q, page_table, max_pages, plan, info.n_kv_heads * info.group, info.group, ws,
+                 status, inverse_fwht, out_bf16, out_f32};
+    if (out_bf16) return launch_fused<true>(fmt, tensor_cores, a, info.n_units, s);
+    return launch_fused<false>(fmt, tensor_cores, a, info.n_units, s);
+}
+
+cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_info &info, int inverse_fwht,
+                           uint16_t *out_bf16, float *out_f32, cudaStream_t s) {
+    const int groups = info.n_seq * info.n_kv_heads;
+    if (groups == 0) return cudaSuccess;
+    combine_kernel<<<groups, 256, 0, s>>>(ws, plan, info.n_kv_heads, info.group, inverse_fwht, out_bf16, out_f32);
+    return cudaGetLastError();
 }
 
 }  // namespace kvq

@@ -97,6 +97,11 @@ __host__ __device__ inline int plan_len_for(int n_units, int n_seq, int n_kv) {
     return PLAN_HEADER + 4 * n_units + n_seq * n_kv + 1;
 }
 __host__ __device__ inline int ws_unit_floats(int G) { return G * D + WS_TAIL; }
+// Workspace = partials of every unit, then one int32 arrival counter per
+// (sequence, KV head) group (used by the fused combine), padded to 16 bytes.
+__host__ __device__ inline uint64_t ws_bytes_for(int n_units, int G, int n_groups) {
+    return (uint64_t)n_units * ws_unit_floats(G) * 4 + (((uint64_t)n_groups * 4 + 15) & ~(uint64_t)15);
+}
 
 // ---------------------------------------------------------------------------
 // PTX helpers
@@ -140,15 +145,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread (up to hint_ns) until the
+// phase completes, instead of returning at once: waiting warps do not spin.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait on an mbarrier phase with a time limit.  Returns false (and the caller
 // records KVQ_STATUS_TIMEOUT) if the phase did not complete within limit_ns.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) return false;
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// 2^x on the special-function unit (inputs <= 0 here; -inf gives +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier.
@@ -214,7 +240,8 @@ cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer
                           const int32_t *page_table, int max_pages, int n_seq, int32_t *status, cudaStream_t s);
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
-                          const kvq_plan_info &info, float *ws, int32_t *status, cudaStream_t s);
+                          const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht,
+                          uint16_t *out_bf16, float *out_f32, cudaStream_t s);
 cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_info &info, int inverse_fwht,
                            uint16_t *out_bf16, float *out_f32, cudaStream_t s);
 

@@ -13,19 +13,28 @@ REL_L2 = 1e-3     # attention output tolerance, fp32 output vs fp64 oracle
 MAX_ABS = 2e-3
 
 
-def decode_step(dw, layer, q, impl="mma", n_ctas=0, status=None):
-    """q: [B, Hq, 256] fp32 device (unrotated).  Returns (out_f32, out_bf16, status, plan, info)."""
+def decode_step(dw, layer, q, impl="mma", n_ctas=0, status=None, mode="split", repeat=1):
+    """q: [B, Hq, 256] fp32 device (unrotated).  mode 'split': decode then
+    attn_combine; 'fused': the *_combined entry point (run `repeat` times on the
+    same workspace).  Returns (out_f32, out_bf16, status, plan, info)."""
     w = dw.w
     plan, info = kvq.decode_plan(dw.pool.desc, dw.seq_lens, dw.page_table.shape[1], n_ctas)
     plan_d = torch.from_numpy(plan).cuda()
-    ws = torch.empty(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
     qp = kvq.q_rotate(q) if kvq.rotated_q(w.fmt) else q
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    kvq.paged_decode_attn(dw.pool, layer, qp, dw.page_table, plan_d, info, ws, status, cudacore=(impl == "alu"))
     out_bf = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
     out_f = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
-    kvq.attn_combine(ws, plan_d, info, kvq.rotated_v(w.fmt), out_bf, out_f)
+    for _ in range(repeat):
+        out_bf.fill_(float("nan"))
+        out_f.fill_(float("nan"))
+        if mode == "fused":
+            kvq.paged_decode_attn_combined(dw.pool, layer, qp, dw.page_table, plan_d, info, ws, out_bf, out_f, status)
+        else:
+            kvq.paged_decode_attn(dw.pool, layer, qp, dw.page_table, plan_d, info, ws, status,
+                                  cudacore=(impl == "alu"))
+            kvq.attn_combine(ws, plan_d, info, kvq.rotated_v(w.fmt), out_bf, out_f)
     torch.cuda.synchronize()
     return out_f.cpu().numpy(), out_bf.cpu(), int(status.item()), plan, info
 

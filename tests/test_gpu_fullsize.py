@@ -40,7 +40,7 @@ def test_full_size_sampled(name):
     q, k, v, pos = kdev.step_inputs(w, [layer])
     import quantized_kv_cache_17_b200 as kvq
     kvq.kv_append(dw.pool, layer, k[0], v[0], pos, dw.page_table)
-    out_f, out_bf, status, plan, info = gc.decode_step(dw, layer, q[0])
+    out_f, out_bf, status, plan, info = gc.decode_step(dw, layer, q[0], mode="fused")
     assert status == 0
     rng = np.random.default_rng(w.seed)
     G = w.group

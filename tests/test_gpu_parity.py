@@ -128,11 +128,12 @@ def _case(name, fmt):
     return w, nctas
 
 
-@pytest.mark.parametrize("impl", ["mma", "alu"])
+@pytest.mark.parametrize("impl", ["mma", "mma_fused", "alu"])
 @pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
 @pytest.mark.parametrize("case", list(CASES))
 def test_decode_matches_oracle(case, fmt, impl):
     w, nctas = _case(case, fmt)
+    mode = "fused" if impl == "mma_fused" else "split"
     dw = kdev.build_pool(w, extra_slots=2)
     q, k, v, pos = kdev.step_inputs(w, [0])
     kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table)          # this step's token
@@ -141,7 +142,8 @@ def test_decode_matches_oracle(case, fmt, impl):
         for g in range(w.n_kv_heads):
             refs[b, g] = gc.oracle_group(dw, 0, b, g)
     for n_ctas in nctas:
-        out_f, out_bf, status, plan, info = gc.decode_step(dw, 0, q[0], impl=impl, n_ctas=n_ctas)
+        out_f, out_bf, status, plan, info = gc.decode_step(dw, 0, q[0], impl=impl.split("_")[0], n_ctas=n_ctas,
+                                                           mode=mode, repeat=2 if mode == "fused" else 1)
         assert status == 0
         G = w.group
         for (b, g), ref in refs.items():

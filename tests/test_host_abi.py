@@ -89,7 +89,8 @@ def _check_plan(plan, info, seq_lens, n_kv, n_ctas):
             assert (us[:, 2] % 64 == 0).all() and (us[:, 3] > us[:, 2]).all()
             assert ((us[:, 3] - us[:, 2]) <= info.chunk_tokens).all()
     G = plan[4]
-    assert info.workspace_bytes == n * (G * 256 + 16) * 4
+    counters = (len(seq_lens) * n_kv * 4 + 15) // 16 * 16
+    assert info.workspace_bytes == n * (G * 256 + 16) * 4 + counters
 
 
 @pytest.mark.parametrize("seq_lens,n_ctas", [([1024], 148), ([262144], 148), ([32768], 148), ([131072], 148),
