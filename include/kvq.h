@@ -207,6 +207,32 @@ int paged_decode_attn_k8v4_combined(const kvq_pool *pool, int layer, const float
                                     uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
                                     void *stream);
 
+/* paged_decode_attn_q4_0_noalloc: paged_decode_attn_q4_0_combined without a
+ * workspace argument, for callers that cannot allocate device memory.  Some
+ * hosts own all device memory and pass a library only the buffers of the call
+ * (a plugin interface of an inference server that forbids allocation while it
+ * runs, to keep memory use fixed, is one); such a caller has nowhere to get the
+ * split-K partial buffer from.  The pages have no counterpart to this entry
+ * point; it is a deployment convenience.
+ *  - Scratch: a file-scope device array of KVQ_NOALLOC_WS_BYTES inside the
+ *    library, held by every GPU that loads the library until the process
+ *    exits.  The plan's info->workspace_bytes must not exceed it (KVQ_ESIZE
+ *    otherwise).
+ *  - The first call on each device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and keeps it; make that first
+ *    call before any stream capture.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree.  Each call clears the
+ *    group arrival counters in the array (cudaMemsetAsync on `stream`) before
+ *    the decode.
+ *  - All calls share the one array: calls that overlap on the GPU (on
+ *    different streams, or from different threads) race and give wrong output.
+ *    Serialise them.
+ * Other arguments and results as paged_decode_attn_q4_0_combined. */
+#define KVQ_NOALLOC_WS_BYTES (8u << 20)
+int paged_decode_attn_q4_0_noalloc(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                   int max_pages, const int32_t *plan, const kvq_plan_info *info, uint16_t *out_bf16,
+                                   float *out_f32, int32_t *status, void *stream);
+
 /* The same computation on CUDA cores only (fp32 FMA, no tensor cores).  Kept
  * as the measured control for the tensor-core kernels above; fmt selects the
  * format. */

@@ -34,7 +34,7 @@ ERRORS = {-1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_EALIGN", -4: "KVQ_E
 EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kvq_decode_plan",
            "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
            "paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined", "paged_decode_attn_k8v4_combined",
-           "paged_decode_attn_cudacore", "attn_combine"]
+           "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine"]
 
 
 class KVQError(RuntimeError):
@@ -86,6 +86,7 @@ def lib():
         for n in ("paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined",
                   "paged_decode_attn_k8v4_combined"):
             getattr(L, n).argtypes = dec[:-2] + [P, P] + dec[-2:]
+        L.paged_decode_attn_q4_0_noalloc.argtypes = dec[:7] + [P, P, P, P]
         L.paged_decode_attn_cudacore.argtypes = [I32] + dec
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
         for n in EXPORTS[1:]:
@@ -179,6 +180,18 @@ def decode_plan(desc: PoolDesc, seq_lens: Sequence[int], max_pages: int, n_ctas:
 
 
 _DECODE = {INT8: "paged_decode_attn_int8", Q4_0: "paged_decode_attn_q4_0", K8V4: "paged_decode_attn_k8v4"}
+NOALLOC_WS_BYTES = 8 << 20
+
+
+def paged_decode_attn_q4_0_noalloc(pool: KVPool, layer: int, q, page_table, plan_dev, info: PlanInfo, out_bf16,
+                                   out_f32=None, status=None, stream=None):
+    """The q4_0 decode with the merge fused in, using the library's own scratch
+    array instead of a caller workspace (for callers that cannot allocate)."""
+    cp = pool.c_pool()
+    _check(lib().paged_decode_attn_q4_0_noalloc(ctypes.byref(cp), layer, _ptr(q), _ptr(page_table),
+                                                page_table.shape[1], _ptr(plan_dev), ctypes.byref(info),
+                                                _ptr(out_bf16), _ptr(out_f32), _ptr(status), _stream(stream)),
+           "paged_decode_attn_q4_0_noalloc")
 
 
 def paged_decode_attn_combined(pool: KVPool, layer: int, q, page_table, plan_dev, info: PlanInfo, workspace,

@@ -30,6 +30,7 @@ SOURCES = {
     "kvq_abi.cu": [],
     "kvq_append.cu": ["-fmad=false"],     # quantiser: no fused multiply-add anywhere in this unit
     "kvq_decode.cu": [],
+    "kvq_noalloc.cu": [],
 }
 
 
