@@ -112,7 +112,7 @@ template <int FMT> struct TcCfg {
     static constexpr int SCALE_WARP = 2 * NQK;
     static constexpr int COPY_WARP = 2 * NQK + 1;
     static constexpr int NTHREADS = (2 * NQK + 2) * 32;
-    static constexpr int ITEMS_PER_STAGE = 4;                   // an item = 2 tiles = 16 tokens
+    static constexpr int ITEMS_PER_STAGE = 2;                   // an item = 4 tiles = 32 tokens
     static constexpr int STAGE_BYTES = 8 * L::BYTES;
     static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
     static constexpr int DP = 4;                                // slots of each QK -> PV ring
@@ -122,7 +122,7 @@ template <int FMT> struct TcCfg {
     static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
     static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
     static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
-    static constexpr int PSLOT = 32 * 4 + 8;                    // floats: p of 32 lanes x 4, alpha[8]
+    static constexpr int PSLOT = 32 * 8 + 8;                    // floats: p of 32 lanes x 8, alpha[8]
     static constexpr int RING = NS * STAGE_BYTES;
     static constexpr int MERGE = (COMBINE_SMEM > 8 * D + 2 * NQK * 8 + 16 ? COMBINE_SMEM : 8 * D + 2 * NQK * 8 + 16) * 4;
     static constexpr int DATA = RING > MERGE ? RING : MERGE;
@@ -242,37 +242,53 @@ template <int FMT> struct QkWarp {
         }
     }
 
-    // Scores, softmax update, and the hand-over slot: p (lane*4 .. +4) and the
-    // rescale factor of head g at [128 + g].
+    // Scores of the four tiles of an item, softmax update, and the hand-over
+    // slot: p of tile j, tokens 2t, 2t+1 at lane*8 + 2j, +1, and the rescale
+    // factor of head g at [256 + g].  The running max keeps one binade of
+    // headroom (it moves to max + 1 only when a score exceeds it), so the rescale
+    // factor is rarely different from 1 and p stays <= 1/2.
     template <bool MASK>
-    __device__ __forceinline__ void item(const uint8_t *tA, const float *fA, int vA, int vB, int lane, float *slot) {
+    __device__ __forceinline__ void item(const uint8_t *tp, const float *fp, const int (&v)[4], int lane,
+                                         float *slot) {
         const int g = lane >> 2, t = lane & 3;
-        float s[4];
-        scores(tA, fA, lane, s);
-        if (MASK) {
-            if (2 * t >= vA) s[0] = -INFINITY;
-            if (2 * t + 1 >= vA) s[1] = -INFINITY;
-            if (2 * t >= vB) s[2] = -INFINITY;
-            if (2 * t + 1 >= vB) s[3] = -INFINITY;
+        float s[8];
+        {
+            float a[4], b[4];
+            scores(tp, fp, lane, a);
+            scores(tp + 2 * L::BYTES, fp + 2 * C::SF_TILE, lane, b);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s[i] = a[i];
+                s[4 + i] = b[i];
+            }
         }
-        float mx = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
+        if (MASK) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (2 * t >= v[j]) s[2 * j] = -INFINITY;
+                if (2 * t + 1 >= v[j]) s[2 * j + 1] = -INFINITY;
+            }
+        }
+        float mx = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3])), fmaxf(fmaxf(s[4], s[5]), fmaxf(s[6], s[7])));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run, mx);       // mx is finite: every item has a valid token
-        const float alpha = ex2(m_run - m_new);      // 1 when the max did not grow; 0 on the first item
+        const float m_new = mx > m_run ? mx + 1.f : m_run;   // mx is finite: every item has a valid token
+        const float alpha = ex2(m_run - m_new);               // 1 when unchanged; 0 on the first item
         l_run *= alpha;
         m_run = m_new;
-        float p[4];
+        float p[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = ex2(s[i] - m_run);
-        l_run += (p[0] + p[1]) + (p[2] + p[3]);
-        sts128(slot + lane * 4, make_uint4(__float_as_uint(p[0]), __float_as_uint(p[1]), __float_as_uint(p[2]),
+        for (int i = 0; i < 8; ++i) p[i] = ex2(s[i] - m_run);
+        l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+        sts128(slot + lane * 8, make_uint4(__float_as_uint(p[0]), __float_as_uint(p[1]), __float_as_uint(p[2]),
                                            __float_as_uint(p[3])));
-        if (t == 0) slot[128 + g] = alpha;
+        sts128(slot + lane * 8 + 4, make_uint4(__float_as_uint(p[4]), __float_as_uint(p[5]), __float_as_uint(p[6]),
+                                               __float_as_uint(p[7])));
+        slot[256 + g] = alpha;          // the four lanes of group g store the same value
     }
     // An item whose page could not be read: nothing to add, nothing to rescale.
     __device__ __forceinline__ void skip(int lane, float *slot) {
-        if (lane < 8) slot[128 + lane] = 1.f;
+        if (lane < 8) slot[256 + lane] = 1.f;
     }
 };
 
@@ -330,23 +346,14 @@ template <int FMT> struct PvWarp {
         }
     }
 
-    // Rescale (factors of heads 2t, 2t+1 from the slot) and accumulate the item.
+    // Tiles A, B (consecutive) with p of their tokens 2t, 2t+1.
     template <bool MASK>
-    __device__ __forceinline__ void item(const uint8_t *tA, int vA, int vB, bool ok, int lane, const float4 &p,
-                                         float2 al) {
-        const int t = lane & 3;
-        if (__any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f)) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                o[i][0] *= al.x; o[i][2] *= al.x;
-                o[i][1] *= al.y; o[i][3] *= al.y;
-            }
-        }
-        if (!ok) return;
+    __device__ __forceinline__ void two_tiles(const uint8_t *tA, int vA, int vB, int t, int lane, float pA0, float pA1,
+                                              float pB0, float pB1) {
         const uint8_t *tB = tA + L::BYTES;
         uint32_t phA, plA, phB, plB;     // p of tokens 2t, 2t+1 as fp16 hi + lo pairs
-        split_pair(p.x, p.y, phA, plA);
-        split_pair(p.z, p.w, phB, plB);
+        split_pair(pA0, pA1, phA, plA);
+        split_pair(pB0, pB1, phB, plB);
         // zero the scales of tokens past the end (their bytes may hold anything)
         const uint32_t mA = MASK ? ((2 * t < vA ? 0xFFFFu : 0u) | (2 * t + 1 < vA ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
         const uint32_t mB = MASK ? ((2 * t < vB ? 0xFFFFu : 0u) | (2 * t + 1 < vB ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
@@ -372,6 +379,24 @@ template <int FMT> struct PvWarp {
                 pv_i8(q, wvA, wvB, u4_at(eA, q) & mA, u4_at(eB, q) & mB, phA, plA, phB, plB);
             }
         }
+    }
+
+    // Rescale (factors of heads 2t, 2t+1 from the slot) and accumulate the four
+    // tiles of an item.
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tp, const int (&v)[4], bool ok, int lane, const float4 &p0,
+                                         const float4 &p1, float2 al) {
+        const int t = lane & 3;
+        if (__any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                o[i][0] *= al.x; o[i][2] *= al.x;
+                o[i][1] *= al.y; o[i][3] *= al.y;
+            }
+        }
+        if (!ok) return;
+        two_tiles<MASK>(tp, v[0], v[1], t, lane, p0.x, p0.y, p0.z, p0.w);
+        two_tiles<MASK>(tp + 2 * L::BYTES, v[2], v[3], t, lane, p1.x, p1.y, p1.z, p1.w);
     }
 
     // Add this warp's o (scaled per head) into o_s[8][256].
@@ -861,7 +886,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     float *wsu = A.ws + (size_t)u * ws_unit_floats(G);
     if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;
     const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
-    const int n_items = (t1 - t0 + 2 * TILE - 1) / (2 * TILE);
+    const int n_items = (t1 - t0 + 4 * TILE - 1) / (4 * TILE);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NS; ++i) {
@@ -903,26 +928,29 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     const int pw = is_qk ? warp : warp - C::NQK;    // pair index
     QkWarp<FMT> qk;
     PvWarp<FMT> pv;
+    // item `it` = tiles 4 it .. 4 it + 3 = half of stage it / 2
     if (is_qk) {
         qk.init(A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D, G, lane);
         int k = 0;
         for (int it = pw; it < n_items; it += C::NQK, ++k) {
-            const int st = (2 * it) >> 3, si = st % C::NS, slot = k % C::DP;
+            const int st = it >> 1, si = st % C::NS, slot = k % C::DP;
             float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
-            if (!mbar_wait_bounded(&full[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
-                !mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
+            // ready implies the stage's bulk copy has landed (the scale warp waited for it)
+            if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
                 (k >= C::DP && !mbar_wait_bounded(&p_empty[pw * C::DP + slot], ((k / C::DP) - 1) & 1, WAIT_LIMIT_NS))) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
-            const int tok = t0 + 2 * it * TILE;
-            const int vA = min(TILE, t1 - tok), vB = max(0, min(TILE, t1 - tok - TILE));
+            const int tok = t0 + it * 4 * TILE;
+            int v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
             if (stage_ok[si]) {
-                const uint8_t *tp = smem + si * C::STAGE_BYTES + ((2 * it) & 7) * L::BYTES;
+                const uint8_t *tp = smem + si * C::STAGE_BYTES + (it & 1) * 4 * L::BYTES;
                 const float *fp = reinterpret_cast<const float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES) +
-                                  ((2 * it) & 7) * C::SF_TILE;
-                if (vA == TILE && vB == TILE) qk.template item<false>(tp, fp, vA, vB, lane, ps);
-                else qk.template item<true>(tp, fp, vA, vB, lane, ps);
+                                  (it & 1) * 4 * C::SF_TILE;
+                if (v[3] == TILE) qk.template item<false>(tp, fp, v, lane, ps);
+                else qk.template item<true>(tp, fp, v, lane, ps);
             } else {
                 qk.skip(lane, ps);
             }
@@ -932,22 +960,24 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         pv.init();
         int k = 0;
         for (int it = pw; it < n_items; it += C::NQK, ++k) {
-            const int st = (2 * it) >> 3, si = st % C::NS, slot = k % C::DP;
+            const int st = it >> 1, si = st % C::NS, slot = k % C::DP;
             const float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
-            if (!mbar_wait_bounded(&p_full[pw * C::DP + slot], (k / C::DP) & 1, WAIT_LIMIT_NS) ||
-                !mbar_wait_bounded(&full[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
+            // p_full implies the QK warp saw the stage ready, hence landed
+            if (!mbar_wait_bounded(&p_full[pw * C::DP + slot], (k / C::DP) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
-            const float4 p = lds128f(ps + lane * 4);
-            const float2 al = make_float2(ps[128 + 2 * (lane & 3)], ps[128 + 2 * (lane & 3) + 1]);
+            const float4 p0 = lds128f(ps + lane * 8), p1 = lds128f(ps + lane * 8 + 4);
+            const float2 al = make_float2(ps[256 + 2 * (lane & 3)], ps[256 + 2 * (lane & 3) + 1]);
             mbar_arrive(&p_empty[pw * C::DP + slot]);
-            const int tok = t0 + 2 * it * TILE;
-            const int vA = min(TILE, t1 - tok), vB = max(0, min(TILE, t1 - tok - TILE));
-            const uint8_t *tp = smem + si * C::STAGE_BYTES + ((2 * it) & 7) * L::BYTES;
+            const int tok = t0 + it * 4 * TILE;
+            int v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
+            const uint8_t *tp = smem + si * C::STAGE_BYTES + (it & 1) * 4 * L::BYTES;
             const bool ok = stage_ok[si] != 0;
-            if (vA == TILE && vB == TILE) pv.template item<false>(tp, vA, vB, ok, lane, p, al);
-            else pv.template item<true>(tp, vA, vB, ok, lane, p, al);
+            if (v[3] == TILE) pv.template item<false>(tp, v, ok, lane, p0, p1, al);
+            else pv.template item<true>(tp, v, ok, lane, p0, p1, al);
             mbar_arrive(&empty[si]);
         }
     }
