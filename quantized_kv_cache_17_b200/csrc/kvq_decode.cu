@@ -77,6 +77,13 @@ __device__ __forceinline__ void mma_acc(float (&d)[4], const uint4 &a, uint32_t 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
+// D = A * B (C = 0), m16n8k8: A = rows g / g+8, k 2t, 2t+1; B = k 2t, 2t+1 of column g.
+__device__ __forceinline__ void mma_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
+}
 __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
@@ -134,7 +141,25 @@ template <int FMT> struct TcCfg {
     static_assert(TOTAL <= 227 * 1024, "shared memory budget");
 };
 
-// Scale warp: convert the fp16 K scales of one stage (8 tiles) to fp32 rows.
+// Scores are formed from the codes as stored (q4_0 nibbles 0..15, int8 codes
+// + 128 as 0..255) placed directly in the low bits of fp16 words: as fp16
+// subnormals they are the exact values code * 2^-24 (or 16 code * 2^-24 for a
+// nibble in bits 4-7), so unpacking costs one AND per two values and no
+// subtraction.  The constant offset (8 or 128) is removed by one extra small
+// MMA per tile: -OFF * sum_b dK[t][b] * Q[b], Q[b] = the query's sum over block
+// b.  Two power-of-two scales keep every fp16 operand in its normal range: the
+// query fragments carry 2^kq (kq puts the group's largest |q| in [2^12, 2^13)),
+// and scores are produced in units of 2^kb, kb = kq - KBS, removed inside the
+// softmax.  The fp32 K scales are therefore stored multiplied by 2^(24 - KBS).
+template <int FMT> struct QkCodes {
+    static constexpr bool Q4 = TileLayout<FMT>::KP == PART_Q4;
+    static constexpr float OFF = Q4 ? 8.f : 128.f;
+    static constexpr int KBS = Q4 ? 6 : 11;
+    static constexpr float KSF = Q4 ? 262144.f : 8192.f;     // 2^(24 - KBS)
+};
+
+// Scale warp: convert the fp16 K scales of one stage (8 tiles) to fp32 rows
+// (times 2^(24 - KBS)).
 template <int FMT>
 __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float *sf, int lane) {
     using L = TileLayout<FMT>;
@@ -142,6 +167,7 @@ __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float
     constexpr int PAIR_B = KSB / 4;                     // 32 (q4) or 16 (i8) bytes per pair
     constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
     constexpr int CPT = KSB / 16;                       // 16-byte chunks per tile
+    constexpr float F = QkCodes<FMT>::KSF;
     for (int c = lane; c < 8 * CPT; c += 32) {
         const int tile = c / CPT, o = (c % CPT) * 16;
         const int pair = o / PAIR_B, within = (o % PAIR_B) / 2;
@@ -149,8 +175,10 @@ __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float
         float *dst = sf + tile * 4 * KSTRIDE + pair * KSTRIDE + within;
         const float2 a = __half22float2(u32_as_h2(h.x)), b = __half22float2(u32_as_h2(h.y));
         const float2 cc = __half22float2(u32_as_h2(h.z)), d = __half22float2(u32_as_h2(h.w));
-        sts128(dst, make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y)));
-        sts128(dst + 4, make_uint4(__float_as_uint(cc.x), __float_as_uint(cc.y), __float_as_uint(d.x), __float_as_uint(d.y)));
+        sts128(dst, make_uint4(__float_as_uint(a.x * F), __float_as_uint(a.y * F), __float_as_uint(b.x * F),
+                               __float_as_uint(b.y * F)));
+        sts128(dst + 4, make_uint4(__float_as_uint(cc.x * F), __float_as_uint(cc.y * F), __float_as_uint(d.x * F),
+                                   __float_as_uint(d.y * F)));
     }
 }
 
@@ -160,38 +188,101 @@ __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float
 template <int FMT> struct QkWarp {
     using L = TileLayout<FMT>;
     using C = TcCfg<FMT>;
-    uint4 qa[16];          // A fragments of the 16 k-steps
+    using K = QkCodes<FMT>;
+    uint4 qa[16];          // A fragments of the 16 k-steps (scaled by 2^kq)
+    uint32_t qb_hi, qb_lo; // A fragment of the offset MMA: -OFF 2^-KBS Q[2t], Q[2t+1] of head g, hi / lo rows
+    float inv_sb;          // 2^-kb
     float m_run, l_run;    // head g (the four lanes of a group agree)
 
-    // Fragment of k-step ks for lane (g, t): rows g (hi) / g+8 (lo) of head g,
-    // dims 16ks + 2t, +1 (a0/a1) and 16ks + 2t + 8, +9 (a2/a3).
-    __device__ static uint4 make_qfrag(const float *qg, int G, int ks, int lane) {
-        const int g = lane >> 2, t = lane & 3;
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (g < G) {
-            const float *p = qg + g * D + 16 * ks + 2 * t;
-            x[0] = p[0] * QSCALE; x[1] = p[1] * QSCALE; x[2] = p[8] * QSCALE; x[3] = p[9] * QSCALE;
-        }
-        uint4 f;
-        split_pair(x[0], x[1], f.x, f.y);
-        split_pair(x[2], x[3], f.z, f.w);
-        return f;
-    }
-
+    // Fragments of head g (rows g: fp16 hi, g+8: fp16 lo), k-step ks: dims
+    // 16ks + 2t, +1 (x, y) and 16ks + 2t + 8, +9 (z, w).  For 4-bit keys the
+    // second pair is divided by 16, matching its codes' 16 code * 2^-24.
     __device__ __forceinline__ void init(const float *qg, int G, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        float mx = 0.f;
+        if (g < G) {
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks) qa[ks] = make_qfrag(qg, G, ks, lane);
+            for (int ks = 0; ks < 16; ++ks) {
+                const float *p = qg + g * D + 16 * ks + 2 * t;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p[0] * QSCALE), fabsf(p[1] * QSCALE)),
+                                     fmaxf(fabsf(p[8] * QSCALE), fabsf(p[9] * QSCALE))));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int kq = 0;
+        if (mx > 0.f) kq = min(max(12 - ((int)((__float_as_uint(mx) >> 23) & 255u) - 127), -60), 60);
+        const float s_lo = __int_as_float((127 + kq) << 23);
+        const float s_hi = K::Q4 ? __int_as_float((127 + kq - 4) << 23) : s_lo;
+        constexpr float M_HI = K::Q4 ? 16.f : 1.f;
+        float S[8];            // sum of the represented query over block b (units 2^kq)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) S[b] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (g < G) {
+                const float *p = qg + g * D + 16 * ks + 2 * t;
+                x[0] = (p[0] * QSCALE) * s_lo; x[1] = (p[1] * QSCALE) * s_lo;
+                x[2] = (p[8] * QSCALE) * s_hi; x[3] = (p[9] * QSCALE) * s_hi;
+            }
+            uint4 f;
+            split_pair(x[0], x[1], f.x, f.y);
+            split_pair(x[2], x[3], f.z, f.w);
+            qa[ks] = f;
+            const float2 h0 = __half22float2(u32_as_h2(f.x)), l0 = __half22float2(u32_as_h2(f.y));
+            const float2 h1 = __half22float2(u32_as_h2(f.z)), l1 = __half22float2(u32_as_h2(f.w));
+            const float r = ((h0.x + l0.x) + (h0.y + l0.y)) + M_HI * ((h1.x + l1.x) + (h1.y + l1.y));
+            S[K::Q4 ? ks >> 1 : ks >> 2] += r;
+        }
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            S[b] += __shfl_xor_sync(0xffffffffu, S[b], 1);
+            S[b] += __shfl_xor_sync(0xffffffffu, S[b], 2);
+        }
+        constexpr float CA = -K::OFF / (float)(1 << K::KBS);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int b = 0; b < 8; b += 2)
+            if (b == 2 * t && (K::Q4 || b < 4)) {
+                a0 = CA * S[b];
+                a1 = CA * S[b + 1];
+            }
+        split_pair(a0, a1, qb_hi, qb_lo);
+        inv_sb = __int_as_float((127 - (kq - K::KBS)) << 23);
         m_run = -INFINITY;
         l_run = 0.f;
     }
 
-    // S[head g][tokens 2t, 2t+1] of tiles A (s[0], s[1]) and B (s[2], s[3]).
+    // B fragment of the offset MMA for one tile: fp16 K scales of token g,
+    // blocks (groups) 2t, 2t+1; zero for the missing groups of int8 keys.
+    __device__ __forceinline__ static uint32_t kscale_frag(const uint8_t *tp, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        if constexpr (K::Q4) {
+            const uint2 w = lds64(tp + L::KS + (g >> 1) * 32 + 8 * t);
+            return __byte_perm(w.x, w.y, (g & 1) ? 0x7632u : 0x5410u);
+        } else {
+            const uint2 w = lds64(tp + L::KS + (g >> 1) * 16 + 8 * (t & 1));
+            return t < 2 ? __byte_perm(w.x, w.y, (g & 1) ? 0x7632u : 0x5410u) : 0u;
+        }
+    }
+
+    // S[head g][tokens 2t, 2t+1] of tiles A (s[0], s[1]) and B (s[2], s[3]), in
+    // units of 2^kb.
     __device__ __forceinline__ void scores(const uint8_t *tA, const float *fA, int lane, float (&s)[4]) const {
         const uint8_t *tB = tA + L::BYTES;
         const float *fB = fA + C::SF_TILE;
         const int t = lane & 3;
-        s[0] = s[1] = s[2] = s[3] = 0.f;
-        if constexpr (L::KP == PART_Q4) {
+        {
+            float ca[4], cb[4];
+            mma_k8(ca, qb_hi, qb_lo, kscale_frag(tA, lane));
+            mma_k8(cb, qb_hi, qb_lo, kscale_frag(tB, lane));
+            s[0] = ca[0] + ca[2];
+            s[1] = ca[1] + ca[3];
+            s[2] = cb[0] + cb[2];
+            s[3] = cb[1] + cb[3];
+        }
+        if constexpr (K::Q4) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const uint4 kA = lds128(tA + L::KC + hf * 512 + lane * 16);
@@ -202,11 +293,12 @@ template <int FMT> struct QkWarp {
                 for (int bb = 0; bb < 4; ++bb) {
                     const int b = 4 * hf + bb;
                     const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
+                    const uint32_t wA2 = wA >> 8, wB2 = wB >> 8;
                     float a[4], c[4];
-                    mma_z(a, qa[2 * b], h2_as_u32(q4_lo_pair(wA)), h2_as_u32(q4_hi_pair(wA)));
-                    mma_z(c, qa[2 * b], h2_as_u32(q4_lo_pair(wB)), h2_as_u32(q4_hi_pair(wB)));
-                    mma_acc(a, qa[2 * b + 1], h2_as_u32(q4_lo_pair(wA >> 8)), h2_as_u32(q4_hi_pair(wA >> 8)));
-                    mma_acc(c, qa[2 * b + 1], h2_as_u32(q4_lo_pair(wB >> 8)), h2_as_u32(q4_hi_pair(wB >> 8)));
+                    mma_z(a, qa[2 * b], wA & 0x000F000Fu, wA & 0x00F000F0u);
+                    mma_z(c, qa[2 * b], wB & 0x000F000Fu, wB & 0x00F000F0u);
+                    mma_acc(a, qa[2 * b + 1], wA2 & 0x000F000Fu, wA2 & 0x00F000F0u);
+                    mma_acc(c, qa[2 * b + 1], wB2 & 0x000F000Fu, wB2 & 0x00F000F0u);
                     const float2 da = f2_at(dA0, dA1, bb), db = f2_at(dB0, dB1, bb);
                     s[0] = fmaf(a[0] + a[2], da.x, s[0]);
                     s[1] = fmaf(a[1] + a[3], da.y, s[1]);
@@ -225,12 +317,14 @@ template <int FMT> struct QkWarp {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint32_t wA = u4_at(kA, j) ^ 0x80808080u, wB = u4_at(kB, j) ^ 0x80808080u;
+                    const uint32_t a0 = __byte_perm(wA, 0u, 0x4140u), a1 = __byte_perm(wA, 0u, 0x4342u);
+                    const uint32_t b0 = __byte_perm(wB, 0u, 0x4140u), b1 = __byte_perm(wB, 0u, 0x4342u);
                     if (j == 0) {
-                        mma_z(a, qa[4 * q], h2_as_u32(i8_pair(wA, 0x4140u)), h2_as_u32(i8_pair(wA, 0x4342u)));
-                        mma_z(c, qa[4 * q], h2_as_u32(i8_pair(wB, 0x4140u)), h2_as_u32(i8_pair(wB, 0x4342u)));
+                        mma_z(a, qa[4 * q], a0, a1);
+                        mma_z(c, qa[4 * q], b0, b1);
                     } else {
-                        mma_acc(a, qa[4 * q + j], h2_as_u32(i8_pair(wA, 0x4140u)), h2_as_u32(i8_pair(wA, 0x4342u)));
-                        mma_acc(c, qa[4 * q + j], h2_as_u32(i8_pair(wB, 0x4140u)), h2_as_u32(i8_pair(wB, 0x4342u)));
+                        mma_acc(a, qa[4 * q + j], a0, a1);
+                        mma_acc(c, qa[4 * q + j], b0, b1);
                     }
                 }
                 const float2 da = f2_at(dA0, dA1, q), db = f2_at(dB0, dB1, q);
@@ -272,13 +366,14 @@ template <int FMT> struct QkWarp {
         float mx = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3])), fmaxf(fmaxf(s[4], s[5]), fmaxf(s[6], s[7])));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx *= inv_sb;                                          // log2 units
         const float m_new = mx > m_run ? mx + 1.f : m_run;   // mx is finite: every item has a valid token
         const float alpha = ex2(m_run - m_new);               // 1 when unchanged; 0 on the first item
         l_run *= alpha;
         m_run = m_new;
         float p[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = ex2(s[i] - m_run);
+        for (int i = 0; i < 8; ++i) p[i] = ex2(fmaf(s[i], inv_sb, -m_run));
         l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         sts128(slot + lane * 8, make_uint4(__float_as_uint(p[0]), __float_as_uint(p[1]), __float_as_uint(p[2]),
                                            __float_as_uint(p[3])));
