@@ -40,7 +40,7 @@ namespace {
 constexpr float QSCALE = 0.09016844005556021f;  // log2(e) / sqrt(256)
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr int COMBINE_MAX_UNITS = 256;            // units per group merged in one pass of the combine
-constexpr int COMBINE_SMEM = 8 * D + 2 * 8 * COMBINE_MAX_UNITS + 16;   // floats of combine scratch
+constexpr int COMBINE_SMEM = 8 * D + 8 * COMBINE_MAX_UNITS + 24;   // floats of combine scratch
 
 __device__ __forceinline__ __half2 q4_lo_pair(uint32_t w) {     // nibbles 0 / 4 of each half -> c - 8
     return __hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(0x64086408u));
@@ -122,16 +122,19 @@ template <int FMT> struct TcCfg {
     static constexpr int ITEMS_PER_STAGE = 2;                   // an item = 4 tiles = 32 tokens
     static constexpr int STAGE_BYTES = 8 * L::BYTES;
     static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
-    static constexpr int DP = 4;                                // slots of each QK -> PV ring
+    static constexpr int DP = 2;                                // slots of each QK -> PV ring
     // fp32 K scales of a stage: per tile, token pair t at float t*KSTRIDE (block
     // or group j of tokens 2t, 2t+1 at 2j, 2j+1); the stride pads rows so the
     // four pairs fall into different banks
     static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
     static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
     static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
-    static constexpr int PSLOT = 32 * 8 + 8;                    // floats: p of 32 lanes x 8, alpha[8]
+    static constexpr int PSLOT = 32 * 8 + 16;                   // floats: p of 32 lanes x 8, alpha[8], item
+    static constexpr int PITEM = 32 * 8 + 8;                    // the item index (int) in a slot
+    static constexpr int OSTRIDE = D + 4;                       // row stride of the PV warps' o buffers
     static constexpr int RING = NS * STAGE_BYTES;
-    static constexpr int MERGE = (COMBINE_SMEM > 8 * D + 2 * NQK * 8 + 16 ? COMBINE_SMEM : 8 * D + 2 * NQK * 8 + 16) * 4;
+    static constexpr int OBUF = NQK * 8 * OSTRIDE + 2 * NQK * 8;   // floats of the CTA merge
+    static constexpr int MERGE = (COMBINE_SMEM > OBUF ? COMBINE_SMEM : OBUF) * 4;
     static constexpr int DATA = RING > MERGE ? RING : MERGE;
     static constexpr int SFOFF = (DATA + 127) & ~127;
     static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
@@ -494,17 +497,17 @@ template <int FMT> struct PvWarp {
         two_tiles<MASK>(tp + 2 * L::BYTES, v[2], v[3], t, lane, p1.x, p1.y, p1.z, p1.w);
     }
 
-    // Add this warp's o (scaled per head) into o_s[8][256].
-    __device__ __forceinline__ void accumulate(float *o_s, const float *scale, int lane) {
+    // Write this warp's o, heads 2t, 2t+1 scaled by sc0, sc1, to b[8][OSTRIDE]
+    // (a row stride of 260 floats keeps the stores of a warp on distinct banks).
+    __device__ __forceinline__ void store_scaled(float *b, float sc0, float sc1, int lane) const {
         const int g = lane >> 2, t = lane & 3;
-        const float sc0 = scale[2 * t], sc1 = scale[2 * t + 1];
+        float *r0 = b + (2 * t) * TcCfg<FMT>::OSTRIDE + g, *r1 = r0 + TcCfg<FMT>::OSTRIDE;
 #pragma unroll
         for (int mt = 0; mt < 16; ++mt) {
-            const int d0 = 16 * mt + g;
-            atomicAdd(o_s + (2 * t) * D + d0, o[mt][0] * sc0);
-            atomicAdd(o_s + (2 * t + 1) * D + d0, o[mt][1] * sc1);
-            atomicAdd(o_s + (2 * t) * D + d0 + 8, o[mt][2] * sc0);
-            atomicAdd(o_s + (2 * t + 1) * D + d0 + 8, o[mt][3] * sc1);
+            r0[16 * mt] = o[mt][0] * sc0;
+            r1[16 * mt] = o[mt][1] * sc1;
+            r0[16 * mt + 8] = o[mt][2] * sc0;
+            r1[16 * mt + 8] = o[mt][3] * sc1;
         }
     }
 };
@@ -719,77 +722,98 @@ template <int FMT, int GT> struct AluCompute {
 // the G output rows starting at out_row.  M = max m_u, L = sum l_u 2^(m_u - M),
 // o = sum 2^(m_u - M) o_u / L, then H/16 if V was stored rotated.  Runs on the
 // first NTH threads of the CTA (named barrier bar_id); sm: COMBINE_SMEM floats.
-// All (m, l) pairs are staged in shared memory first, so the loads of the
-// partial outputs are independent of each other and issue back to back.
+// Warp h computes head h's weights from all units' (m, l) at once (warp max
+// and sum); then every lane keeps 2 UB independent 16-byte loads in flight.
 // ---------------------------------------------------------------------------
 template <int NTH>
 __device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t out_row, int inverse_fwht,
                               uint16_t *out_bf16, float *out_f32, float *sm, int bar_id) {
     constexpr int NWARP = NTH / 32;
+    static_assert(NWARP >= 8, "the weight pass takes one warp per head");
+    constexpr int UB = 8;                         // units whose loads are in flight together (16 float4 / lane)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int stride = ws_unit_floats(G);
     float *o_s = sm;                              // [8][256] accumulated outputs
     float *f_s = sm + 8 * D;                      // [units][8] weights 2^(m_u - M)
-    float *l_s = f_s + 8 * COMBINE_MAX_UNITS;     // [units][8] sums l_u
-    float *Ms = l_s + 8 * COMBINE_MAX_UNITS;      // [8]
-    float *Ls = Ms + 8;                           // [8]
+    float *Ms = f_s + 8 * COMBINE_MAX_UNITS;      // [8] running max
+    float *Ls = Ms + 8;                           // [8] running sum
+    float *Cs = Ls + 8;                           // [8] factor for what is accumulated so far
     for (int i = tid; i < 8 * D; i += NTH) o_s[i] = 0.f;
-    if (tid < 8) {
-        Ms[tid] = -INFINITY;
-        Ls[tid] = 0.f;
-    }
     for (int c0 = u0; c0 < u1; c0 += COMBINE_MAX_UNITS) {     // chunks of units (one pass in practice)
         const int n = min(COMBINE_MAX_UNITS, u1 - c0);
-        // stage m and l of every (unit, head)
-        for (int i = tid; i < n * 8; i += NTH) {
-            const int uu = i >> 3, h = i & 7;
-            const float *p = ws + (size_t)(c0 + uu) * stride + G * D;
-            f_s[i] = h < G ? __ldcg(p + h) : -INFINITY;
-            l_s[i] = h < G ? __ldcg(p + 8 + h) : 0.f;
-        }
-        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
-        // new running max per head; rescale what is accumulated so far
-        if (tid < 8) {
-            float M = Ms[tid];
-            for (int uu = 0; uu < n; ++uu) M = fmaxf(M, f_s[uu * 8 + tid]);
-            const float scale_old = Ms[tid] == -INFINITY ? 0.f : exp2f(Ms[tid] - M);
-            float L = Ls[tid] * scale_old;
-            for (int uu = 0; uu < n; ++uu) {
-                const float m = f_s[uu * 8 + tid];
-                const float f = m == -INFINITY ? 0.f : exp2f(m - M);
-                f_s[uu * 8 + tid] = f;
-                L = fmaf(l_s[uu * 8 + tid], f, L);
-            }
-            l_s[tid] = scale_old;            // reuse: factor for the accumulators of this head
-            Ms[tid] = M;
-            Ls[tid] = L;
-        }
-        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
-        // rescale earlier chunks (only with more than COMBINE_MAX_UNITS units)
-        if (c0 > u0 && warp == 0)
-            for (int h = 0; h < G; ++h)
+        // weights: warp h reads (m, l) of every unit for head h, all loads first
+        if (warp < G) {
+            const int h = warp;
+            float m[COMBINE_MAX_UNITS / 32], l[COMBINE_MAX_UNITS / 32];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o_s[h * D + lane * 8 + i] *= l_s[h];
+            for (int j = 0; j < COMBINE_MAX_UNITS / 32; ++j) {
+                const int uu = lane + 32 * j;
+                const float *p = ws + (size_t)(c0 + uu) * stride + G * D;
+                m[j] = uu < n ? __ldcg(p + h) : -INFINITY;
+                l[j] = uu < n ? __ldcg(p + 8 + h) : 0.f;
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < COMBINE_MAX_UNITS / 32; ++j) M = fmaxf(M, m[j]);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            const float M_old = c0 == u0 ? -INFINITY : Ms[h];
+            M = fmaxf(M, M_old);
+            float L = 0.f;
+#pragma unroll
+            for (int j = 0; j < COMBINE_MAX_UNITS / 32; ++j) {
+                const float f = m[j] == -INFINITY ? 0.f : exp2f(m[j] - M);
+                if (lane + 32 * j < n) f_s[(lane + 32 * j) * 8 + h] = f;
+                L = fmaf(l[j], f, L);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            __syncwarp();
+            if (lane == 0) {
+                const float c = M_old == -INFINITY ? 0.f : exp2f(M_old - M);
+                Cs[h] = c;
+                Ls[h] = (c0 == u0 ? 0.f : Ls[h] * c) + L;
+                Ms[h] = M;
+            }
+        }
         asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
-        // warps per head: warp w takes head w % G and every wph-th unit; the unit
-        // loads are independent of each other (weights come from shared memory)
-        const int wph = NWARP >= G ? NWARP / G : 1;
+        if (c0 > u0) {                                  // rescale earlier chunks
+            for (int i = tid; i < G * D; i += NTH) o_s[i] *= Cs[i >> 8];
+            asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+        }
+        // warps per head: warp w takes head w % G and every wph-th unit, UB units
+        // (2 UB independent 16-byte loads per lane) at a time
+        const int wph = NWARP / G;
         if (warp < wph * G) {
             const int h = warp % G, part = warp / G;
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int uu = part; uu < n; uu += wph) {
-                const float f = f_s[uu * 8 + h];
-                const float *p = ws + (size_t)(c0 + uu) * stride + h * D + lane * 8;
-                const float4 a = __ldcg(reinterpret_cast<const float4 *>(p));
-                const float4 b = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
-                acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
-                acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
-                acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
-                acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
-            }
+            for (int ub = part; ub < n; ub += UB * wph) {
+                float4 a[UB], b[UB];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) atomicAdd(o_s + h * D + lane * 8 + i, acc[i]);
+                for (int j = 0; j < UB; ++j) {
+                    const int uu = ub + j * wph;
+                    const float4 *p = reinterpret_cast<const float4 *>(ws + (size_t)(c0 + min(uu, n - 1)) * stride +
+                                                                       h * D + lane * 8);
+                    a[j] = __ldcg(p);
+                    b[j] = __ldcg(p + 1);
+                }
+#pragma unroll
+                for (int j = 0; j < UB; ++j) {
+                    const int uu = ub + j * wph;
+                    const float f = uu < n ? f_s[uu * 8 + h] : 0.f;
+                    acc[0] = fmaf(a[j].x, f, acc[0]); acc[1] = fmaf(a[j].y, f, acc[1]);
+                    acc[2] = fmaf(a[j].z, f, acc[2]); acc[3] = fmaf(a[j].w, f, acc[3]);
+                    acc[4] = fmaf(b[j].x, f, acc[4]); acc[5] = fmaf(b[j].y, f, acc[5]);
+                    acc[6] = fmaf(b[j].z, f, acc[6]); acc[7] = fmaf(b[j].w, f, acc[7]);
+                }
+            }
+            if (wph == 1) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o_s[h * D + lane * 8 + i] += acc[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) atomicAdd(o_s + h * D + lane * 8 + i, acc[i]);
+            }
         }
         asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
     }
@@ -916,26 +940,14 @@ __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, ui
     }
 }
 
-// After the warps' states are in m_s/l_s [n_rep][8] and o_s [8][256] (scaled to
-// M_s): write the unit's partial; with FUSED, the last CTA of the (sequence, KV
-// head) group merges the group.  Runs on the NCT merge threads (bar 1).
+// The unit's partial is in the workspace: with FUSED, count the unit in and let
+// the last CTA of the (sequence, KV head) group merge the group.  Runs on the
+// NCT merge threads (bar 1).
 template <bool FUSED, int NCT>
-__device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_s, const float *m_s, const float *l_s,
-                                            const float *M_s, int n_rep, float *wsu, int seq, int kvh, int n_units,
-                                            int *s_last, uint8_t *smem) {
-    const int G = A.G;
-    for (int i = threadIdx.x; i < G * D; i += NCT) wsu[i] = o_s[i];
-    if (threadIdx.x < 8) {
-        const int h = threadIdx.x;
-        float Lh = 0.f;
-        for (int w = 0; w < n_rep; ++w) {
-            const float mw = m_s[w * 8 + h];
-            if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M_s[h]);
-        }
-        wsu[G * D + h] = M_s[h];
-        wsu[G * D + 8 + h] = Lh;
-    }
+__device__ __forceinline__ void publish_unit(const DecodeArgs &A, int seq, int kvh, int n_units, int *s_last,
+                                             uint8_t *smem) {
     if constexpr (FUSED) {
+        const int G = A.G;
         const int32_t *start = A.plan + PLAN_HEADER + 4 * n_units;
         const int grp = seq * A.geo.n_kv_heads + kvh;
         int *counter = reinterpret_cast<int *>(A.ws + (size_t)n_units * ws_unit_floats(G)) + grp;
@@ -954,6 +966,27 @@ __device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_
                                A.inverse_fwht, A.out_bf16, A.out_f32, reinterpret_cast<float *>(smem), 1);
         }
     }
+}
+
+// After the warps' states are in m_s/l_s [n_rep][8] and o_s [8][256] (scaled to
+// M_s): write the unit's partial, then publish it.
+template <bool FUSED, int NCT>
+__device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_s, const float *m_s, const float *l_s,
+                                            const float *M_s, int n_rep, float *wsu, int seq, int kvh, int n_units,
+                                            int *s_last, uint8_t *smem) {
+    const int G = A.G;
+    for (int i = threadIdx.x; i < G * D; i += NCT) wsu[i] = o_s[i];
+    if (threadIdx.x < 8) {
+        const int h = threadIdx.x;
+        float Lh = 0.f;
+        for (int w = 0; w < n_rep; ++w) {
+            const float mw = m_s[w * 8 + h];
+            if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M_s[h]);
+        }
+        wsu[G * D + h] = M_s[h];
+        wsu[G * D + 8 + h] = Lh;
+    }
+    publish_unit<FUSED, NCT>(A, seq, kvh, n_units, s_last, smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -1023,16 +1056,28 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     const int pw = is_qk ? warp : warp - C::NQK;    // pair index
     QkWarp<FMT> qk;
     PvWarp<FMT> pv;
-    // item `it` = tiles 4 it .. 4 it + 3 = half of stage it / 2
+    // Pair pw takes items pw, pw + NQK, ... (item `it` = tiles 4 it .. 4 it + 3 =
+    // half of stage it / 2); the QK warp passes the item index, or -1 at the end,
+    // to its PV warp with the scores.  (Handing items out from a shared counter
+    // instead measured slower on long units.)
     if (is_qk) {
         qk.init(A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D, G, lane);
-        int k = 0;
-        for (int it = pw; it < n_items; it += C::NQK, ++k) {
-            const int st = it >> 1, si = st % C::NS, slot = k % C::DP;
+        for (int k = 0;; ++k) {
+            const int slot = k % C::DP;
             float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
+            if (k >= C::DP && !mbar_wait_bounded(&p_empty[pw * C::DP + slot], ((k / C::DP) - 1) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            const int it = pw + C::NQK * k;
+            if (it >= n_items) {                       // no work left: tell the PV warp
+                if (lane == 0) reinterpret_cast<int *>(ps)[C::PITEM] = -1;
+                mbar_arrive(&p_full[pw * C::DP + slot]);
+                break;
+            }
+            const int st = it >> 1, si = st % C::NS;
             // ready implies the stage's bulk copy has landed (the scale warp waited for it)
-            if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS) ||
-                (k >= C::DP && !mbar_wait_bounded(&p_empty[pw * C::DP + slot], ((k / C::DP) - 1) & 1, WAIT_LIMIT_NS))) {
+            if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
@@ -1049,22 +1094,25 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
             } else {
                 qk.skip(lane, ps);
             }
+            if (lane == 0) reinterpret_cast<int *>(ps)[C::PITEM] = it;
             mbar_arrive(&p_full[pw * C::DP + slot]);
         }
     } else {
         pv.init();
-        int k = 0;
-        for (int it = pw; it < n_items; it += C::NQK, ++k) {
-            const int st = it >> 1, si = st % C::NS, slot = k % C::DP;
+        for (int k = 0;; ++k) {
+            const int slot = k % C::DP;
             const float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
             // p_full implies the QK warp saw the stage ready, hence landed
             if (!mbar_wait_bounded(&p_full[pw * C::DP + slot], (k / C::DP) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
+            const int it = reinterpret_cast<const int *>(ps)[C::PITEM];
+            if (it < 0) break;
             const float4 p0 = lds128f(ps + lane * 8), p1 = lds128f(ps + lane * 8 + 4);
             const float2 al = make_float2(ps[256 + 2 * (lane & 3)], ps[256 + 2 * (lane & 3) + 1]);
             mbar_arrive(&p_empty[pw * C::DP + slot]);
+            const int st = it >> 1, si = st % C::NS;
             const int tok = t0 + it * 4 * TILE;
             int v[4];
 #pragma unroll
@@ -1077,13 +1125,13 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         }
     }
 
-    // ---- CTA merge: QK warps report (m, l), PV warps add o ---------------------
+    // ---- CTA merge: QK warps report (m, l); PV warps write o scaled to the CTA
+    // max into their own buffer; the merge threads sum the buffers into the
+    // partial -----------------------------------------------------------------
     asm volatile("bar.sync 1, %0;" ::"r"(NCT));               // every consumer is done with the ring
-    float *o_s = reinterpret_cast<float *>(smem);             // [8][256]
-    float *m_s = o_s + 8 * D;                                 // [NQK][8]
+    float *obuf = reinterpret_cast<float *>(smem);            // [NQK][8][OSTRIDE]
+    float *m_s = obuf + C::NQK * 8 * C::OSTRIDE;              // [NQK][8]
     float *l_s = m_s + C::NQK * 8;                            // [NQK][8]
-    float *M_s = l_s + C::NQK * 8;                            // [8]
-    for (int i = threadIdx.x; i < 8 * D; i += NCT) o_s[i] = 0.f;
     if (is_qk) {
         float lr = qk.l_run;
         lr += __shfl_xor_sync(0xffffffffu, lr, 1);
@@ -1094,23 +1142,40 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(NCT));
-    if (threadIdx.x < 8) {
-        float M = -INFINITY;
-        for (int w = 0; w < C::NQK; ++w) M = fmaxf(M, m_s[w * 8 + threadIdx.x]);
-        M_s[threadIdx.x] = M;
-    }
-    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
     if (!is_qk) {
-        float scale[8];
+        const int t = lane & 3;
+        float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            const float mw = m_s[pw * 8 + h];
-            scale[h] = mw == -INFINITY ? 0.f : exp2f(mw - M_s[h]);
+        for (int w = 0; w < C::NQK; ++w) {
+            M0 = fmaxf(M0, m_s[w * 8 + 2 * t]);
+            M1 = fmaxf(M1, m_s[w * 8 + 2 * t + 1]);
         }
-        pv.accumulate(o_s, scale, lane);
+        const float m0 = m_s[pw * 8 + 2 * t], m1 = m_s[pw * 8 + 2 * t + 1];
+        const float sc0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0), sc1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
+        pv.store_scaled(obuf + pw * 8 * C::OSTRIDE, sc0, sc1, lane);
+    } else if (warp == 0 && lane < 8) {
+        const int h = lane;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) M = fmaxf(M, m_s[w * 8 + h]);
+        float Lh = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) {
+            const float mw = m_s[w * 8 + h];
+            if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M);
+        }
+        wsu[G * D + h] = M;
+        wsu[G * D + 8 + h] = Lh;
     }
     asm volatile("bar.sync 1, %0;" ::"r"(NCT));
-    finish_unit<FUSED, NCT>(A, o_s, m_s, l_s, M_s, C::NQK, wsu, seq, kvh, n_units, &s_last, smem);
+    for (int i = threadIdx.x; i < G * D; i += NCT) {
+        const float *b = obuf + (i >> 8) * C::OSTRIDE + (i & 255);
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) acc += b[w * 8 * C::OSTRIDE];
+        wsu[i] = acc;
+    }
+    publish_unit<FUSED, NCT>(A, seq, kvh, n_units, &s_last, smem);
 }
 
 // ---------------------------------------------------------------------------

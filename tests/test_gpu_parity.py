@@ -117,6 +117,9 @@ CASES = {
     "ragged_g6": (small("q4_0", 24, 4, [1, 77, 300, 1025], outlier="student_t", q_post=1 / 16,
                         q_outliers=False, n_out=8), [0, 5]),
     "ragged_g8": (small("q4_0", 16, 2, [513, 64, 8]), [0, 2]),
+    # 300 steps split 300 ways: more units in one group than the merge takes in one pass
+    "many_units_300": (small("q4_0", 6, 1, [19200], outlier="student_t", q_post=1 / 16, q_outliers=False, n_out=8),
+                       [300]),
 }
 
 
