@@ -717,6 +717,48 @@ template <int FMT, int GT> struct AluCompute {
     }
 };
 
+// One output row (256 dims, lane holds dims 8 lane .. 8 lane + 7, already
+// divided by L): H/16 if V was stored rotated (butterflies inside the lane for
+// the low three index bits, then across lanes), then fp32 and bf16 stores.
+__device__ __forceinline__ void finish_row(float (&x)[8], int lane, int inverse_fwht, int64_t row, uint16_t *out_bf16,
+                                           float *out_f32) {
+    if (inverse_fwht) {
+#pragma unroll
+        for (int hh = 1; hh < 8; hh <<= 1)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if ((i & hh) == 0) {
+                    const float a = x[i], b = x[i + hh];
+                    x[i] = a + b;
+                    x[i + hh] = a - b;
+                }
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float other = __shfl_xor_sync(0xffffffffu, x[i], m);
+                x[i] = upper ? other - x[i] : x[i] + other;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] *= 0.0625f;
+    }
+    const size_t off = (size_t)row * D + lane * 8;
+    if (out_f32) {
+        float4 *o = reinterpret_cast<float4 *>(out_f32 + off);
+        o[0] = make_float4(x[0], x[1], x[2], x[3]);
+        o[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        pk[i] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    *reinterpret_cast<uint4 *>(out_bf16 + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+}
+
 // ---------------------------------------------------------------------------
 // Merge of one (sequence, KV head) group: units [u0, u1) of the workspace ->
 // the G output rows starting at out_row.  M = max m_u, L = sum l_u 2^(m_u - M),
@@ -823,41 +865,110 @@ __device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t ou
         const float inv = 1.0f / Ls[h];
 #pragma unroll
         for (int i = 0; i < 8; ++i) x[i] = o_s[h * D + lane * 8 + i] * inv;
-        if (inverse_fwht) {
+        finish_row(x, lane, inverse_fwht, out_row + h, out_bf16, out_f32);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of head h of one (sequence, KV head) group by one CTA, used when every
+// CTA of the launch is resident at once (cooperative launch): each CTA of the
+// group takes its own heads, so the group's partials are read by up to G CTAs
+// in parallel instead of by the last one alone.  Units [u0, u0 + n); NTH
+// threads (named barrier bar_id); sm: MH_SMEM floats.
+// ---------------------------------------------------------------------------
+constexpr int MH_MAX_UNITS = 256;                 // units per group on this path
+constexpr int MH_BATCH = 8;                       // float4 loads in flight per thread
+template <int NTH>
+__device__ void merge_head(const float *ws, int G, int u0, int n, int h, int64_t out_row, int inverse_fwht,
+                           uint16_t *out_bf16, float *out_f32, float *sm, int bar_id) {
+    constexpr int NPART = NTH / 64;               // threads per float4 column of the head
+    static_assert(NPART >= 1 && NTH % 64 == 0, "threads");
+    const int tid = threadIdx.x, lane = tid & 31, c = tid & 63, part = tid >> 6;
+    const int stride = ws_unit_floats(G);
+    float *f_s = sm;                              // [n] weights 2^(m_u - M)
+    float *red = f_s + MH_MAX_UNITS;              // [NPART][256] partial sums
+    float *o_s = red + NPART * D;                 // [256]
+    float *L_s = o_s + D;                         // [1]
+    const float *base = ws + (size_t)u0 * stride + h * D + 4 * c;
+    // first batch of this thread's loads, issued before the weights are known
+    float4 v[MH_BATCH];
 #pragma unroll
-            for (int hh = 1; hh < 8; hh <<= 1)
+    for (int j = 0; j < MH_BATCH; ++j) {
+        const int uu = part + j * NPART;
+        v[j] = uu < n ? __ldcg(reinterpret_cast<const float4 *>(base + (size_t)uu * stride)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < 32) {
+        float m[MH_MAX_UNITS / 32], l[MH_MAX_UNITS / 32];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if ((i & hh) == 0) {
-                        const float a = x[i], b = x[i + hh];
-                        x[i] = a + b;
-                        x[i + hh] = a - b;
-                    }
-#pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const bool upper = (lane & m) != 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float other = __shfl_xor_sync(0xffffffffu, x[i], m);
-                    x[i] = upper ? other - x[i] : x[i] + other;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] *= 0.0625f;
+        for (int j = 0; j < MH_MAX_UNITS / 32; ++j) {
+            const int uu = lane + 32 * j;
+            const float *p = ws + (size_t)(u0 + uu) * stride + G * D;
+            m[j] = uu < n ? __ldcg(p + h) : -INFINITY;
+            l[j] = uu < n ? __ldcg(p + 8 + h) : 0.f;
         }
-        const size_t off = (size_t)(out_row + h) * D + lane * 8;
-        if (out_f32) {
-            float4 *o = reinterpret_cast<float4 *>(out_f32 + off);
-            o[0] = make_float4(x[0], x[1], x[2], x[3]);
-            o[1] = make_float4(x[4], x[5], x[6], x[7]);
-        }
-        uint32_t pk[4];
+        float M = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-            pk[i] = *reinterpret_cast<const uint32_t *>(&v);
+        for (int j = 0; j < MH_MAX_UNITS / 32; ++j) M = fmaxf(M, m[j]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+#pragma unroll
+        for (int j = 0; j < MH_MAX_UNITS / 32; ++j) {
+            const float f = m[j] == -INFINITY ? 0.f : exp2f(m[j] - M);
+            if (lane + 32 * j < n) f_s[lane + 32 * j] = f;
+            L = fmaf(l[j], f, L);
         }
-        *reinterpret_cast<uint4 *>(out_bf16 + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) *L_s = L;
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b0 = 0;; b0 += MH_BATCH * NPART) {
+#pragma unroll
+        for (int j = 0; j < MH_BATCH; ++j) {
+            const int uu = b0 + part + j * NPART;
+            const float f = uu < n ? f_s[uu] : 0.f;
+            acc.x = fmaf(v[j].x, f, acc.x); acc.y = fmaf(v[j].y, f, acc.y);
+            acc.z = fmaf(v[j].z, f, acc.z); acc.w = fmaf(v[j].w, f, acc.w);
+        }
+        if (b0 + MH_BATCH * NPART >= n) break;
+#pragma unroll
+        for (int j = 0; j < MH_BATCH; ++j) {
+            const int uu = b0 + MH_BATCH * NPART + part + j * NPART;
+            v[j] = uu < n ? __ldcg(reinterpret_cast<const float4 *>(base + (size_t)uu * stride)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    reinterpret_cast<float4 *>(red + part * D)[c] = acc;
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+    for (int i = tid; i < D; i += NTH) {
+        float s = 0.f;
+#pragma unroll
+        for (int p = 0; p < NPART; ++p) s += red[p * D + i];
+        o_s[i] = s;
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+    if (tid < 32) {
+        float x[8];
+        const float inv = 1.0f / *L_s;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = o_s[lane * 8 + i] * inv;
+        finish_row(x, lane, inverse_fwht, out_row + h, out_bf16, out_f32);
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
+}
+
+// Spin (with a time limit) until *p >= target; acquire ordering on success.
+__device__ __forceinline__ bool wait_count_at_least(const int *p, int target, uint64_t limit_ns) {
+    uint64_t t0 = 0;
+    for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > limit_ns) return false;
+        __nanosleep(128);
     }
 }
 
@@ -876,6 +987,7 @@ struct DecodeArgs {
     int inverse_fwht;      // fused combine: un-rotate the output
     uint16_t *out_bf16;    // fused combine outputs (NULL: write partials only)
     float *out_f32;
+    int coop;              // fused combine: every CTA is resident (cooperative launch); merge heads in parallel
 };
 
 // ---------------------------------------------------------------------------
@@ -953,6 +1065,27 @@ __device__ __forceinline__ void publish_unit(const DecodeArgs &A, int seq, int k
         int *counter = reinterpret_cast<int *>(A.ws + (size_t)n_units * ws_unit_floats(G)) + grp;
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+        if (A.coop) {
+            // every CTA of the group counts in, waits for the others, merges its
+            // heads (rank, rank + n_grp, ...) and counts out; the last one out
+            // resets the counter for the next launch
+            const int n_grp = start[grp + 1] - start[grp];
+            if (threadIdx.x == 0) {
+                atomicAdd(counter, 1);
+                *s_last = wait_count_at_least(counter, n_grp, WAIT_LIMIT_NS);
+                if (!*s_last) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                __threadfence();
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+            if (*s_last) {
+                const int64_t row0 = (int64_t)seq * A.n_q_heads + (int64_t)kvh * G;
+                for (int h = blockIdx.x - start[grp]; h < G; h += n_grp)
+                    merge_head<NCT>(A.ws, G, start[grp], n_grp, h, row0, A.inverse_fwht, A.out_bf16, A.out_f32,
+                                    reinterpret_cast<float *>(smem), 1);
+            }
+            if (threadIdx.x == 0 && atomicAdd(counter, 1) == 2 * n_grp - 1) *counter = 0;
+            return;
+        }
         if (threadIdx.x == 0) {
             const int n_grp = start[grp + 1] - start[grp];
             const int old = atomicAdd(counter, 1);
@@ -1290,15 +1423,47 @@ cudaError_t launch_k(K kernel, int smem_bytes, int threads, const DecodeArgs &a,
         if (e != cudaSuccess) return e;
         configured = true;
     }
+    if (a.coop) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(n_units);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem_bytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kernel, a);
+    }
     kernel<<<n_units, threads, smem_bytes, s>>>(a);
     return cudaGetLastError();
+}
+
+// CTAs of `kernel` that can be resident at once on the current device.
+template <typename K>
+int resident_ctas(K kernel, int smem_bytes, int threads) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem_bytes) != cudaSuccess) return 0;
+    return sms * per_sm;
 }
 
 template <int FMT, bool FUSED>
 cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s) {
     if (tc) {
         static bool cfg = false;
-        return launch_k(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS, a, n_units, s, cfg);
+        DecodeArgs b = a;
+        if (FUSED) {
+            static int cap[64] = {};     // resident CTAs per device ordinal (0: not yet known)
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+            if (cap[dev] == 0) cap[dev] = resident_ctas(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS);
+            b.coop = n_units <= cap[dev] && n_units <= MH_MAX_UNITS ? 1 : 0;
+        }
+        return launch_k(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS, b, n_units, s, cfg);
     }
     static bool c4 = false, c6 = false, c8 = false;
     switch (a.G) {
@@ -1324,7 +1489,7 @@ cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const
                           const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht, uint16_t *out_bf16,
                           float *out_f32, cudaStream_t s) {
     DecodeArgs a{pool, geo, layer, q, page_table, max_pages, plan, info.n_kv_heads * info.group, info.group, ws,
-                 status, inverse_fwht, out_bf16, out_f32};
+                 status, inverse_fwht, out_bf16, out_f32, 0};
     if (out_bf16) return launch_fused<true>(fmt, tensor_cores, a, info.n_units, s);
     return launch_fused<false>(fmt, tensor_cores, a, info.n_units, s);
 }
