@@ -122,24 +122,25 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def cpu_oracle_rate(fmt: str, G: int, codes_list, qp_list, budget_s: float):
-    """Time the oracle (single thread, as it stands) on the given (layer, KV
-    head) groups; returns (KV GB/s, token-kvheads/s, seconds, groups done)."""
+def cpu_oracle_rate(fmt: str, G: int, groups, budget_s: float):
+    """Time the oracle (single thread, as it stands) on (layer, KV head) groups;
+    `groups` yields ((kc, ks, vc, vs), qp) and only the oracle calls are timed.
+    Returns (KV GB/s, token-kvheads/s, seconds, groups done)."""
     import oracle
-    t0 = time.perf_counter()
+    dt = 0.0
     done_bytes = 0
     done_tok = 0
     n = 0
     per_tok = oracle.format_bytes_per_token_head(fmt)
-    for codes, qp in zip(codes_list, qp_list):
-        kc, ks, vc, vs = codes
+    for (kc, ks, vc, vs), qp in groups:
+        t0 = time.perf_counter()
         oracle.attn_decode(fmt, qp, kc, ks, vc, vs)
+        dt += time.perf_counter() - t0
         done_tok += kc.shape[0]
         done_bytes += kc.shape[0] * per_tok
         n += 1
-        if time.perf_counter() - t0 > budget_s:
+        if dt > budget_s:
             break
-    dt = time.perf_counter() - t0
     return done_bytes / dt / 1e9, done_tok / dt, dt, n
 
 
@@ -349,13 +350,14 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         from tests import kvq_layout
-        codes_list, qp_list = [], []
-        for g in range(min(args.cpu_groups, w.n_kv_heads)):
+        def groups():
             b = len(w.seq_lens) - 1
-            codes_list.append(kvq_layout.gather_sequence(fmt, dw.pool.buf, layout, L - 1, g, dw.page_table_host[b],
-                                                         w.seq_lens[b]))
-            qp_list.append(oracle.q_prepare(fmt, q[L - 1, b, g * w.group:(g + 1) * w.group].cpu().numpy()))
-        gbs, tok_rate, dt, n = cpu_oracle_rate(fmt, w.group, codes_list, qp_list, args.cpu_budget)
+            for idx in range(min(args.cpu_groups, L * w.n_kv_heads)):
+                lay, g = L - 1 - idx // w.n_kv_heads, idx % w.n_kv_heads   # last layers first
+                codes = kvq_layout.gather_sequence(fmt, dw.pool.buf, layout, lay, g, dw.page_table_host[b],
+                                                   w.seq_lens[b])
+                yield codes, oracle.q_prepare(fmt, q[lay, b, g * w.group:(g + 1) * w.group].cpu().numpy())
+        gbs, tok_rate, dt, n = cpu_oracle_rate(fmt, w.group, groups(), args.cpu_budget)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"oracle fp64 attention of {n} (layer, KV head) groups ({w.group} query heads each) over "
                          f"{w.seq_lens[-1]} tokens of {w.name}, codes read back from the GPU pool; "
@@ -408,7 +410,7 @@ def main():
     ap.add_argument("--no-fuse", action="store_true", help="separate attn_combine launch")
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-groups", type=int, default=4)
+    ap.add_argument("--cpu-groups", type=int, default=16)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     if args.warmup < 3:
