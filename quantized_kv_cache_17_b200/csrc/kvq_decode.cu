@@ -119,7 +119,8 @@ template <int FMT> struct TcCfg {
     static constexpr int SCALE_WARP = 2 * NQK;
     static constexpr int COPY_WARP = 2 * NQK + 1;
     static constexpr int NTHREADS = (2 * NQK + 2) * 32;
-    static constexpr int ITEMS_PER_STAGE = 2;                   // an item = 4 tiles = 32 tokens
+    static constexpr int TPI = FMT == KVQ_INT8 ? 2 : 4;         // tiles per work item (measured best)
+    static constexpr int ITEMS_PER_STAGE = 8 / TPI;
     static constexpr int STAGE_BYTES = 8 * L::BYTES;
     static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
     static constexpr int DP = 2;                                // slots of each QK -> PV ring
@@ -129,8 +130,9 @@ template <int FMT> struct TcCfg {
     static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
     static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
     static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
-    static constexpr int PSLOT = 32 * 8 + 16;                   // floats: p of 32 lanes x 8, alpha[8], item
-    static constexpr int PITEM = 32 * 8 + 8;                    // the item index (int) in a slot
+    static constexpr int PA = 32 * 2 * TPI;                     // alpha[8] in a slot, after p of 32 lanes x 2 TPI
+    static constexpr int PSLOT = PA + 16;                       // floats: p, alpha[8], item
+    static constexpr int PITEM = PA + 8;                        // the item index (int) in a slot
     static constexpr int OSTRIDE = D + 4;                       // row stride of the PV warps' o buffers
     static constexpr int RING = NS * STAGE_BYTES;
     static constexpr int OBUF = NQK * 8 * OSTRIDE + 2 * NQK * 8;   // floats of the CTA merge
@@ -339,34 +341,34 @@ template <int FMT> struct QkWarp {
         }
     }
 
-    // Scores of the four tiles of an item, softmax update, and the hand-over
-    // slot: p of tile j, tokens 2t, 2t+1 at lane*8 + 2j, +1, and the rescale
-    // factor of head g at [256 + g].  The running max keeps one binade of
+    // Scores of the TPI tiles of an item, softmax update, and the hand-over
+    // slot: p of tile j, tokens 2t, 2t+1 at lane*2TPI + 2j, +1, and the rescale
+    // factor of head g at [PA + g].  The running max keeps one binade of
     // headroom (it moves to max + 1 only when a score exceeds it), so the rescale
     // factor is rarely different from 1 and p stays <= 1/2.
     template <bool MASK>
-    __device__ __forceinline__ void item(const uint8_t *tp, const float *fp, const int (&v)[4], int lane,
+    __device__ __forceinline__ void item(const uint8_t *tp, const float *fp, const int (&v)[C::TPI], int lane,
                                          float *slot) {
+        constexpr int NS2 = 2 * C::TPI;       // scores per lane: tokens 2t, 2t+1 of each tile
         const int g = lane >> 2, t = lane & 3;
-        float s[8];
-        {
-            float a[4], b[4];
-            scores(tp, fp, lane, a);
-            scores(tp + 2 * L::BYTES, fp + 2 * C::SF_TILE, lane, b);
+        float s[NS2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                s[i] = a[i];
-                s[4 + i] = b[i];
-            }
+        for (int h = 0; h < C::TPI / 2; ++h) {
+            float a[4];
+            scores(tp + 2 * h * L::BYTES, fp + 2 * h * C::SF_TILE, lane, a);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[4 * h + i] = a[i];
         }
         if (MASK) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < C::TPI; ++j) {
                 if (2 * t >= v[j]) s[2 * j] = -INFINITY;
                 if (2 * t + 1 >= v[j]) s[2 * j + 1] = -INFINITY;
             }
         }
-        float mx = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3])), fmaxf(fmaxf(s[4], s[5]), fmaxf(s[6], s[7])));
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < NS2; ++i) mx = fmaxf(mx, s[i]);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         mx *= inv_sb;                                          // log2 units
@@ -374,19 +376,22 @@ template <int FMT> struct QkWarp {
         const float alpha = ex2(m_run - m_new);               // 1 when unchanged; 0 on the first item
         l_run *= alpha;
         m_run = m_new;
-        float p[8];
+        float p[NS2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = ex2(fmaf(s[i], inv_sb, -m_run));
-        l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        sts128(slot + lane * 8, make_uint4(__float_as_uint(p[0]), __float_as_uint(p[1]), __float_as_uint(p[2]),
-                                           __float_as_uint(p[3])));
-        sts128(slot + lane * 8 + 4, make_uint4(__float_as_uint(p[4]), __float_as_uint(p[5]), __float_as_uint(p[6]),
-                                               __float_as_uint(p[7])));
-        slot[256 + g] = alpha;          // the four lanes of group g store the same value
+        for (int i = 0; i < NS2; ++i) p[i] = ex2(fmaf(s[i], inv_sb, -m_run));
+        float ls = 0.f;
+#pragma unroll
+        for (int i = 0; i < NS2; i += 4) {
+            ls += (p[i] + p[i + 1]) + (p[i + 2] + p[i + 3]);
+            sts128(slot + lane * NS2 + i, make_uint4(__float_as_uint(p[i]), __float_as_uint(p[i + 1]),
+                                                     __float_as_uint(p[i + 2]), __float_as_uint(p[i + 3])));
+        }
+        l_run += ls;
+        slot[C::PA + g] = alpha;        // the four lanes of group g store the same value
     }
     // An item whose page could not be read: nothing to add, nothing to rescale.
     __device__ __forceinline__ void skip(int lane, float *slot) {
-        if (lane < 8) slot[256 + lane] = 1.f;
+        if (lane < 8) slot[C::PA + lane] = 1.f;
     }
 };
 
@@ -482,8 +487,8 @@ template <int FMT> struct PvWarp {
     // Rescale (factors of heads 2t, 2t+1 from the slot) and accumulate the four
     // tiles of an item.
     template <bool MASK>
-    __device__ __forceinline__ void item(const uint8_t *tp, const int (&v)[4], bool ok, int lane, const float4 &p0,
-                                         const float4 &p1, float2 al) {
+    __device__ __forceinline__ void item(const uint8_t *tp, const int (&v)[TcCfg<FMT>::TPI], bool ok, int lane,
+                                         const float4 (&pv)[TcCfg<FMT>::TPI / 2], float2 al) {
         const int t = lane & 3;
         if (__any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f)) {
 #pragma unroll
@@ -493,8 +498,9 @@ template <int FMT> struct PvWarp {
             }
         }
         if (!ok) return;
-        two_tiles<MASK>(tp, v[0], v[1], t, lane, p0.x, p0.y, p0.z, p0.w);
-        two_tiles<MASK>(tp + 2 * L::BYTES, v[2], v[3], t, lane, p1.x, p1.y, p1.z, p1.w);
+#pragma unroll
+        for (int h = 0; h < TcCfg<FMT>::TPI / 2; ++h)
+            two_tiles<MASK>(tp + 2 * h * L::BYTES, v[2 * h], v[2 * h + 1], t, lane, pv[h].x, pv[h].y, pv[h].z, pv[h].w);
     }
 
     // Write this warp's o, heads 2t, 2t+1 scaled by sc0, sc1, to b[8][OSTRIDE]
@@ -1147,7 +1153,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     float *wsu = A.ws + (size_t)u * ws_unit_floats(G);
     if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;
     const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
-    const int n_items = (t1 - t0 + 4 * TILE - 1) / (4 * TILE);
+    const int n_items = (t1 - t0 + C::TPI * TILE - 1) / (C::TPI * TILE);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NS; ++i) {
@@ -1208,21 +1214,21 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
                 mbar_arrive(&p_full[pw * C::DP + slot]);
                 break;
             }
-            const int st = it >> 1, si = st % C::NS;
+            const int st = it / C::ITEMS_PER_STAGE, si = st % C::NS, within = it % C::ITEMS_PER_STAGE;
             // ready implies the stage's bulk copy has landed (the scale warp waited for it)
             if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
-            const int tok = t0 + it * 4 * TILE;
-            int v[4];
+            const int tok = t0 + it * C::TPI * TILE;
+            int v[C::TPI];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
+            for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
             if (stage_ok[si]) {
-                const uint8_t *tp = smem + si * C::STAGE_BYTES + (it & 1) * 4 * L::BYTES;
+                const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
                 const float *fp = reinterpret_cast<const float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES) +
-                                  (it & 1) * 4 * C::SF_TILE;
-                if (v[3] == TILE) qk.template item<false>(tp, fp, v, lane, ps);
+                                  within * C::TPI * C::SF_TILE;
+                if (v[C::TPI - 1] == TILE) qk.template item<false>(tp, fp, v, lane, ps);
                 else qk.template item<true>(tp, fp, v, lane, ps);
             } else {
                 qk.skip(lane, ps);
@@ -1242,18 +1248,20 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
             }
             const int it = reinterpret_cast<const int *>(ps)[C::PITEM];
             if (it < 0) break;
-            const float4 p0 = lds128f(ps + lane * 8), p1 = lds128f(ps + lane * 8 + 4);
-            const float2 al = make_float2(ps[256 + 2 * (lane & 3)], ps[256 + 2 * (lane & 3) + 1]);
-            mbar_arrive(&p_empty[pw * C::DP + slot]);
-            const int st = it >> 1, si = st % C::NS;
-            const int tok = t0 + it * 4 * TILE;
-            int v[4];
+            float4 pp[C::TPI / 2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
-            const uint8_t *tp = smem + si * C::STAGE_BYTES + (it & 1) * 4 * L::BYTES;
+            for (int h = 0; h < C::TPI / 2; ++h) pp[h] = lds128f(ps + lane * 2 * C::TPI + 4 * h);
+            const float2 al = make_float2(ps[C::PA + 2 * (lane & 3)], ps[C::PA + 2 * (lane & 3) + 1]);
+            mbar_arrive(&p_empty[pw * C::DP + slot]);
+            const int st = it / C::ITEMS_PER_STAGE, si = st % C::NS, within = it % C::ITEMS_PER_STAGE;
+            const int tok = t0 + it * C::TPI * TILE;
+            int v[C::TPI];
+#pragma unroll
+            for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
+            const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
             const bool ok = stage_ok[si] != 0;
-            if (v[3] == TILE) pv.template item<false>(tp, v, ok, lane, p0, p1, al);
-            else pv.template item<true>(tp, v, ok, lane, p0, p1, al);
+            if (v[C::TPI - 1] == TILE) pv.template item<false>(tp, v, ok, lane, pp, al);
+            else pv.template item<true>(tp, v, ok, lane, pp, al);
             mbar_arrive(&empty[si]);
         }
     }
@@ -1286,7 +1294,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         const float m0 = m_s[pw * 8 + 2 * t], m1 = m_s[pw * 8 + 2 * t + 1];
         const float sc0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0), sc1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
         pv.store_scaled(obuf + pw * 8 * C::OSTRIDE, sc0, sc1, lane);
-    } else if (warp == 0 && lane < 8) {
+    } else if (pw == 0 && lane < 8) {
         const int h = lane;
         float M = -INFINITY;
 #pragma unroll
