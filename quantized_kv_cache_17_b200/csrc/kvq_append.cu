@@ -52,6 +52,7 @@ __device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
 }
 
 __global__ void __launch_bounds__(128) q_rotate_kernel(const float *q, float *q_rot, int64_t n_vec) {
+    grid_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t vec = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (vec >= n_vec) return;
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(128) append_kernel(uint8_t *pool, PoolGeom geo
                                                      const int32_t *row_pos, const int32_t *page_table,
                                                      int max_pages, int n_seq, int32_t *status) {
     using L = TileLayout<FMT>;
+    grid_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     const int64_t row = item / geo.n_kv_heads;
@@ -258,8 +260,7 @@ __global__ void __launch_bounds__(128) append_kernel(uint8_t *pool, PoolGeom geo
 cudaError_t launch_q_rotate(const float *q, float *q_rot, int64_t n_vec, cudaStream_t s) {
     if (n_vec == 0) return cudaSuccess;
     const int64_t blocks = (n_vec + 3) / 4;
-    q_rotate_kernel<<<(unsigned)blocks, 128, 0, s>>>(q, q_rot, n_vec);
-    return cudaGetLastError();
+    return launch_ex(q_rotate_kernel, dim3((unsigned)blocks), dim3(128), 0, s, false, q, q_rot, n_vec);
 }
 
 cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer, const float *k,
@@ -268,21 +269,10 @@ cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer
     if (n_rows == 0) return cudaSuccess;
     const int64_t items = n_rows * geo.n_kv_heads;
     const unsigned blocks = (unsigned)((items + 3) / 4);
-    switch (fmt) {
-    case KVQ_INT8:
-        append_kernel<KVQ_INT8><<<blocks, 128, 0, s>>>(pool, geo, layer, k, v, n_rows, row_seq, row_pos,
-                                                       page_table, max_pages, n_seq, status);
-        break;
-    case KVQ_Q4_0:
-        append_kernel<KVQ_Q4_0><<<blocks, 128, 0, s>>>(pool, geo, layer, k, v, n_rows, row_seq, row_pos,
-                                                       page_table, max_pages, n_seq, status);
-        break;
-    default:
-        append_kernel<KVQ_K8V4><<<blocks, 128, 0, s>>>(pool, geo, layer, k, v, n_rows, row_seq, row_pos,
-                                                       page_table, max_pages, n_seq, status);
-        break;
-    }
-    return cudaGetLastError();
+    auto kern = fmt == KVQ_INT8 ? append_kernel<KVQ_INT8> : (fmt == KVQ_Q4_0 ? append_kernel<KVQ_Q4_0>
+                                                                                : append_kernel<KVQ_K8V4>);
+    return launch_ex(kern, dim3(blocks), dim3(128), 0, s, false, pool, geo, layer, k, v, n_rows, row_seq, row_pos,
+                     page_table, max_pages, n_seq, status);
 }
 
 }  // namespace kvq

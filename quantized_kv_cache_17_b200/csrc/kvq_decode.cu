@@ -1144,6 +1144,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     int *stage_ok = reinterpret_cast<int *>(p_empty + C::NQK * C::DP);
     __shared__ int s_last;
 
+    grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.x;
     const int32_t *U = A.plan + PLAN_HEADER + 4 * u;
@@ -1339,6 +1340,7 @@ __global__ void __launch_bounds__(AluCfg<FMT>::NTHREADS, 1) decode_alu_kernel(co
     using L = TileLayout<FMT>;
     using C = AluCfg<FMT>;
     extern __shared__ __align__(128) uint8_t smem[];
+    grid_dependency_wait();
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *empty = full + C::NS;
     int *stage_ok = reinterpret_cast<int *>(empty + C::NS);
@@ -1415,6 +1417,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       int n_kv, int G, int inverse_fwht, uint16_t *out_bf16,
                                                       float *out_f32) {
     __shared__ float sm[COMBINE_SMEM];
+    grid_dependency_wait();
     const int grp = blockIdx.x;
     const int seq = grp / n_kv, kvh = grp - seq * n_kv;
     const int n_units = plan[1];
@@ -1431,21 +1434,7 @@ cudaError_t launch_k(K kernel, int smem_bytes, int threads, const DecodeArgs &a,
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (a.coop) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(n_units);
-        cfg.blockDim = dim3(threads);
-        cfg.dynamicSmemBytes = smem_bytes;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, kernel, a);
-    }
-    kernel<<<n_units, threads, smem_bytes, s>>>(a);
-    return cudaGetLastError();
+    return launch_ex(kernel, dim3(n_units), dim3(threads), smem_bytes, s, a.coop != 0, a);
 }
 
 // CTAs of `kernel` that can be resident at once on the current device.
@@ -1506,8 +1495,8 @@ cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_
                            uint16_t *out_bf16, float *out_f32, cudaStream_t s) {
     const int groups = info.n_seq * info.n_kv_heads;
     if (groups == 0) return cudaSuccess;
-    combine_kernel<<<groups, 256, 0, s>>>(ws, plan, info.n_kv_heads, info.group, inverse_fwht, out_bf16, out_f32);
-    return cudaGetLastError();
+    return launch_ex(combine_kernel, dim3(groups), dim3(256), 0, s, false, ws, plan, info.n_kv_heads, info.group,
+                     inverse_fwht, out_bf16, out_f32);
 }
 
 }  // namespace kvq

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -88,6 +89,31 @@ struct PoolGeom {
     int n_pages, n_kv_heads;
 };
 
+// Launch with programmatic stream serialisation (and, with coop, as a
+// cooperative launch: every block resident at once).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool coop,
+                      Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (coop) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // Plan (int32): [magic, n_units, n_seq, n_kv_heads, group, chunk, 0, 0]
 //               units[n_units][4] = {seq, kv_head, t_begin, t_end}
@@ -169,6 +195,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
+
+// Programmatic dependent launch: every kernel of the library is launched with
+// programmatic stream serialisation, so its launch overlaps the exit of the
+// previous kernel in the stream; it then waits here, before reading anything
+// that kernel may have written, until that kernel has completed and its writes
+// are visible.  (No kernel signals early completion, so a dependent kernel
+// starts only as the previous one's blocks exit.)  A no-op for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // 2^x on the special-function unit (inputs <= 0 here; -inf gives +0).
 __device__ __forceinline__ float ex2(float x) {
