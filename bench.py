@@ -223,10 +223,11 @@ def run_ours(args):
 
     def layer_step(l):
         qq = q[l]
-        if rot_q:
-            kvq.q_rotate(qq, q_rot[l])
+        if rot_q:       # q_rotate and kv_append in one launch
+            kvq.kv_append_q_rotate(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, qq, q_rot[l], status=status)
             qq = q_rot[l]
-        kvq.kv_append(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, status=status)
+        else:
+            kvq.kv_append(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, status=status)
         if fused:
             kvq.paged_decode_attn_combined(dw.pool, l, qq, dw.page_table, plan_d, info, ws, out_bf[l], out_f[l],
                                            status)
@@ -247,7 +248,7 @@ def run_ours(args):
             else:
                 kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, cudacore=use_alu)
 
-    launches_per_layer = (2 if fused else 3) + (1 if rot_q else 0)
+    launches_per_layer = 2 if fused else 3      # (kv_append[_q_rotate], decode[, combine])
 
     def barrier():
         if dist is not None:

@@ -137,6 +137,17 @@ int kv_append(const kvq_pool *pool, int layer, const float *k, const float *v, i
               const int32_t *row_seq, const int32_t *row_pos, const int32_t *page_table,
               int max_pages, int n_seq, int32_t *status, void *stream);
 
+/* kv_append_q_rotate: kv_append (arguments as there) and q_rotate of n_vec
+ * query vectors (q -> q_rot, device [n_vec][256] fp32, may alias) in one kernel
+ * launch.  The results are bit-identical to the two separate calls; the only
+ * difference is one launch fewer per decode step.  Either part may be empty
+ * (n_rows == 0 or n_vec == 0).  The pages have no such combined call: it
+ * merges the two steps that precede the decode. */
+int kv_append_q_rotate(const kvq_pool *pool, int layer, const float *k, const float *v, int64_t n_rows,
+                       const int32_t *row_seq, const int32_t *row_pos, const int32_t *page_table,
+                       int max_pages, int n_seq, const float *q, float *q_rot, int64_t n_vec,
+                       int32_t *status, void *stream);
+
 /* Split plan for a batch of sequences (host only).  A plan partitions every
  * (sequence, KV head) token range into work units of whole 64-token steps so
  * that the number of units does not exceed n_ctas (0 = 2 per SM of the current

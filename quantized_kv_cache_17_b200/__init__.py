@@ -31,7 +31,8 @@ STATUS_BAD_SLOT, STATUS_BAD_PLAN, STATUS_TIMEOUT = 1, 2, 4
 ERRORS = {-1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_EALIGN", -4: "KVQ_ECUDA", -5: "KVQ_ESIZE"}
 
 # entry points declared in include/kvq.h
-EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kvq_decode_plan",
+EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kv_append_q_rotate",
+           "kvq_decode_plan",
            "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
            "paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined", "paged_decode_attn_k8v4_combined",
            "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine"]
@@ -79,6 +80,7 @@ def lib():
         L.kvq_pool_layout.argtypes = [ctypes.POINTER(PoolDesc), ctypes.POINTER(Layout)]
         L.q_rotate.argtypes = [P, P, I64, P]
         L.kv_append.argtypes = [ctypes.POINTER(Pool), I32, P, P, I64, P, P, P, I32, I32, P, P]
+        L.kv_append_q_rotate.argtypes = [ctypes.POINTER(Pool), I32, P, P, I64, P, P, P, I32, I32, P, P, I64, P, P]
         L.kvq_decode_plan.argtypes = [ctypes.POINTER(PoolDesc), I32, P, I32, I32, P, I32, ctypes.POINTER(PlanInfo)]
         dec = [ctypes.POINTER(Pool), I32, P, P, I32, P, ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P]
         for n in ("paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4"):
@@ -163,6 +165,20 @@ def kv_append(pool: KVPool, layer: int, k, v, row_pos, page_table, row_seq=None,
     cp = pool.c_pool()
     _check(lib().kv_append(ctypes.byref(cp), layer, _ptr(k), _ptr(v), n_rows, _ptr(row_seq), _ptr(row_pos),
                            _ptr(page_table), max_pages, n_seq, _ptr(status), _stream(stream)), "kv_append")
+
+
+def kv_append_q_rotate(pool: KVPool, layer: int, k, v, row_pos, page_table, q, q_rot=None, row_seq=None,
+                       status=None, stream=None):
+    """kv_append of rows k, v and q_rotate of q ([..., 256] fp32) in one launch; returns q_rot."""
+    if q_rot is None:
+        q_rot = q.new_empty(q.shape)
+    n_rows = 0 if k is None else k.shape[0]
+    n_seq, max_pages = page_table.shape
+    cp = pool.c_pool()
+    _check(lib().kv_append_q_rotate(ctypes.byref(cp), layer, _ptr(k), _ptr(v), n_rows, _ptr(row_seq), _ptr(row_pos),
+                                    _ptr(page_table), max_pages, n_seq, _ptr(q), _ptr(q_rot), q.numel() // HEAD_DIM,
+                                    _ptr(status), _stream(stream)), "kv_append_q_rotate")
+    return q_rot
 
 
 def decode_plan(desc: PoolDesc, seq_lens: Sequence[int], max_pages: int, n_ctas: int = 0):

@@ -132,6 +132,26 @@ int kv_append(const kvq_pool *pool, int layer, const float *k, const float *v, i
                                  static_cast<cudaStream_t>(stream)));
 }
 
+int kv_append_q_rotate(const kvq_pool *pool, int layer, const float *k, const float *v, int64_t n_rows,
+                       const int32_t *row_seq, const int32_t *row_pos, const int32_t *page_table, int max_pages,
+                       int n_seq, const float *q, float *q_rot, int64_t n_vec, int32_t *status, void *stream) {
+    PoolGeom geo;
+    int rc = check_pool(pool, layer, &geo);
+    if (rc) return rc;
+    if (n_rows < 0 || n_vec < 0 || max_pages <= 0 || n_seq <= 0) return KVQ_EINVAL;
+    if (n_rows == 0 && n_vec == 0) return KVQ_OK;
+    if (n_rows > 0 && (!k || !v || !row_pos || !page_table)) return KVQ_EINVAL;
+    if (n_vec > 0 && (!q || !q_rot)) return KVQ_EINVAL;
+    if ((n_rows > 0 && (!aligned16(k) || !aligned16(v))) || (n_vec > 0 && (!aligned16(q) || !aligned16(q_rot))))
+        return KVQ_EALIGN;
+    if ((int64_t)max_pages * PAGE > INT32_MAX || n_rows * geo.n_kv_heads > ((int64_t)1 << 34) ||
+        n_vec > ((int64_t)1 << 34))
+        return KVQ_EINVAL;
+    return cuda_rc(launch_append_rotate(pool->desc.fmt, static_cast<uint8_t *>(pool->base), geo, layer, k, v, n_rows,
+                                        row_seq, row_pos, page_table, max_pages, n_seq, status, q, q_rot, n_vec,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len, int max_pages, int n_ctas,
                     int32_t *plan, int plan_capacity, kvq_plan_info *info) {
     int rc = check_desc(desc);

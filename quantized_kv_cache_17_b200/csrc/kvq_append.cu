@@ -51,17 +51,20 @@ __device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
     x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
-__global__ void __launch_bounds__(128) q_rotate_kernel(const float *q, float *q_rot, int64_t n_vec) {
-    grid_dependency_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t vec = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (vec >= n_vec) return;
+// One warp rotates query vector `vec` of 256 values.
+__device__ __forceinline__ void rotate_vec(const float *q, float *q_rot, int64_t vec, int lane) {
     float x[8];
     load8(q + vec * D + lane * 8, x);
     fwht256_lane(x, lane);
     float4 *o = reinterpret_cast<float4 *>(q_rot + vec * D + lane * 8);
     o[0] = make_float4(x[0], x[1], x[2], x[3]);
     o[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+
+__global__ void __launch_bounds__(128) q_rotate_kernel(const float *q, float *q_rot, int64_t n_vec) {
+    grid_dependency_wait();
+    const int64_t vec = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (vec < n_vec) rotate_vec(q, q_rot, vec, threadIdx.x & 31);
 }
 
 // ---- q4_0: blocks of 32 = 4 lanes (lanes 4b .. 4b+3 hold block b) ----------
@@ -198,15 +201,13 @@ __device__ __forceinline__ void store_scale_i8(uint8_t *sc, int r, int lane, __h
         *reinterpret_cast<__half *>(sc + (r >> 1) * 16 + (lane >> 3) * 4 + (r & 1) * 2) = d;
 }
 
+// One warp encodes (row, KV head) `item`.
 template <int FMT>
-__global__ void __launch_bounds__(128) append_kernel(uint8_t *pool, PoolGeom geo, int layer, const float *k,
-                                                     const float *v, int64_t n_rows, const int32_t *row_seq,
-                                                     const int32_t *row_pos, const int32_t *page_table,
-                                                     int max_pages, int n_seq, int32_t *status) {
+__device__ __forceinline__ void append_item(uint8_t *pool, const PoolGeom &geo, int layer, const float *k,
+                                            const float *v, int64_t n_rows, const int32_t *row_seq,
+                                            const int32_t *row_pos, const int32_t *page_table, int max_pages,
+                                            int n_seq, int32_t *status, int64_t item, int lane) {
     using L = TileLayout<FMT>;
-    grid_dependency_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     const int64_t row = item / geo.n_kv_heads;
     const int head = (int)(item - row * geo.n_kv_heads);
     if (row >= n_rows) return;
@@ -255,12 +256,55 @@ __global__ void __launch_bounds__(128) append_kernel(uint8_t *pool, PoolGeom geo
     }
 }
 
+template <int FMT>
+__global__ void __launch_bounds__(128) append_kernel(uint8_t *pool, PoolGeom geo, int layer, const float *k,
+                                                     const float *v, int64_t n_rows, const int32_t *row_seq,
+                                                     const int32_t *row_pos, const int32_t *page_table,
+                                                     int max_pages, int n_seq, int32_t *status) {
+    grid_dependency_wait();
+    append_item<FMT>(pool, geo, layer, k, v, n_rows, row_seq, row_pos, page_table, max_pages, n_seq, status,
+                     (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5), threadIdx.x & 31);
+}
+
+// kv_append and q_rotate of one decode step in one launch: blocks below
+// append_blocks encode (row, KV head) items, the rest rotate query vectors.
+template <int FMT>
+__global__ void __launch_bounds__(128) append_rotate_kernel(uint8_t *pool, PoolGeom geo, int layer, const float *k,
+                                                            const float *v, int64_t n_rows, const int32_t *row_seq,
+                                                            const int32_t *row_pos, const int32_t *page_table,
+                                                            int max_pages, int n_seq, int32_t *status,
+                                                            unsigned append_blocks, const float *q, float *q_rot,
+                                                            int64_t n_vec) {
+    grid_dependency_wait();
+    const int lane = threadIdx.x & 31;
+    if (blockIdx.x < append_blocks) {
+        append_item<FMT>(pool, geo, layer, k, v, n_rows, row_seq, row_pos, page_table, max_pages, n_seq, status,
+                         (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5), lane);
+    } else {
+        const int64_t vec = (int64_t)(blockIdx.x - append_blocks) * 4 + (threadIdx.x >> 5);
+        if (vec < n_vec) rotate_vec(q, q_rot, vec, lane);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_q_rotate(const float *q, float *q_rot, int64_t n_vec, cudaStream_t s) {
     if (n_vec == 0) return cudaSuccess;
     const int64_t blocks = (n_vec + 3) / 4;
     return launch_ex(q_rotate_kernel, dim3((unsigned)blocks), dim3(128), 0, s, false, q, q_rot, n_vec);
+}
+
+cudaError_t launch_append_rotate(int fmt, uint8_t *pool, const PoolGeom &geo, int layer, const float *k,
+                                 const float *v, int64_t n_rows, const int32_t *row_seq, const int32_t *row_pos,
+                                 const int32_t *page_table, int max_pages, int n_seq, int32_t *status, const float *q,
+                                 float *q_rot, int64_t n_vec, cudaStream_t s) {
+    const int64_t items = n_rows * geo.n_kv_heads;
+    const unsigned ablocks = (unsigned)((items + 3) / 4), rblocks = (unsigned)((n_vec + 3) / 4);
+    if (ablocks + rblocks == 0) return cudaSuccess;
+    auto kern = fmt == KVQ_INT8 ? append_rotate_kernel<KVQ_INT8>
+                                : (fmt == KVQ_Q4_0 ? append_rotate_kernel<KVQ_Q4_0> : append_rotate_kernel<KVQ_K8V4>);
+    return launch_ex(kern, dim3(ablocks + rblocks), dim3(128), 0, s, false, pool, geo, layer, k, v, n_rows, row_seq,
+                     row_pos, page_table, max_pages, n_seq, status, ablocks, q, q_rot, n_vec);
 }
 
 cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer, const float *k,

@@ -191,3 +191,23 @@ def test_decode_bad_plan_reports_status():
     kvq.paged_decode_attn(dw.pool, 0, q[0], dw.page_table, plan_d, info, ws, status)
     torch.cuda.synchronize()
     assert int(status.item()) & kvq.STATUS_BAD_PLAN
+
+
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+def test_kv_append_q_rotate_matches_separate_calls(fmt):
+    """The combined launch writes the same pool bytes and the same rotated query."""
+    w = small(fmt, 12, 2, [300, 513])
+    a = kdev.build_pool(w, prefill_last=False)
+    b = kdev.build_pool(w, prefill_last=False)
+    q, k, v, pos = kdev.step_inputs(w, [0])
+    kvq.kv_append(a.pool, 0, k[0], v[0], pos, a.page_table)
+    qa = kvq.q_rotate(q[0])
+    qb = kvq.kv_append_q_rotate(b.pool, 0, k[0], v[0], pos, b.page_table, q[0])
+    torch.cuda.synchronize()
+    assert torch.equal(a.pool.buf, b.pool.buf)
+    assert torch.equal(qa.view(torch.int32), qb.view(torch.int32))
+    want = oracle.fwht256_f32(q[0].cpu().numpy().reshape(-1, 256))
+    assert np.array_equal(qb.cpu().numpy().reshape(-1, 256).view(np.uint32), want.view(np.uint32))
+    qc = kvq.kv_append_q_rotate(b.pool, 0, None, None, pos, b.page_table, q[0])    # rotation only
+    torch.cuda.synchronize()
+    assert torch.equal(qc.view(torch.int32), qa.view(torch.int32))
