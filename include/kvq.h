@@ -150,8 +150,8 @@ int kv_append_q_rotate(const kvq_pool *pool, int layer, const float *k, const fl
 
 /* Split plan for a batch of sequences (host only).  A plan partitions every
  * (sequence, KV head) token range into work units of whole 64-token steps so
- * that the number of units does not exceed n_ctas (0 = 2 per SM of the current
- * device) and units are as even as possible; it also records, per
+ * that the number of units does not exceed n_ctas (0 = one per SM of the
+ * current device) and units are as even as possible; it also records, per
  * (sequence, KV head), the first unit.  seq_len: host int32 [n_seq], the
  * attended length of each sequence including this step's token, 1 <=
  * seq_len <= max_pages*256.  plan: host int32 array of plan_capacity entries,
@@ -200,11 +200,20 @@ int paged_decode_attn_k8v4(const kvq_pool *pool, int layer, const float *q, cons
                            uint64_t workspace_bytes, int32_t *status, void *stream);
 
 /* paged_decode_attn_<fmt>_combined: the same decode with attn_combine fused
- * into it.  The last CTA to finish a (sequence, KV head) group (counted with an
- * atomic counter in the workspace, never a wait) merges the group's partials,
- * un-rotates (q4_0, k8v4) and writes out_bf16 / out_f32 exactly as
- * attn_combine would.  Saves the combine launch; otherwise identical contract.
- * Calls on the same workspace must not overlap on the GPU. */
+ * into it; out_bf16 / out_f32 are written exactly as attn_combine would (merge,
+ * un-rotation for q4_0 and k8v4).  Saves the combine launch; otherwise the
+ * same contract.  How the group merge runs:
+ *  - When every CTA of the launch can be resident at once (info->n_units not
+ *    above what the device holds; the default plan has one unit per SM), the
+ *    launch is cooperative.  The CTAs of a (sequence, KV head) group count
+ *    themselves in on the group's counter in the workspace and wait for one
+ *    another (2 s limit; past it KVQ_STATUS_TIMEOUT and no output for the
+ *    group).  CTA r of the group then merges heads r, r + n, ... of it.
+ *  - Otherwise the last CTA of a group to finish, found with the same counter
+ *    (no wait), merges the whole group.
+ * Every call leaves the counters at zero, except after a TIMEOUT status: then
+ * zero-fill them again.  Calls on the same workspace must not overlap on the
+ * GPU. */
 int paged_decode_attn_int8_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                                     int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                                     uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
