@@ -122,6 +122,23 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+def max_over_ranks(dist, values, device="cpu"):
+    """Element-wise max of per-rank timings over all ranks (the values as they
+    are with one process).  Every rank must call it, in the same order."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_gbs(world: int, bytes_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job GB/s when every rank streams the same bytes per step
+    (independent replicas) and a step takes ms_per_step (max over ranks)."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def cpu_oracle_rate(fmt: str, G: int, groups, budget_s: float):
     """Time the oracle (single thread, as it stands) on (layer, KV head) groups;
     `groups` yields ((kc, ks, vc, vs), qp) and only the oracle calls are timed.
@@ -332,15 +349,12 @@ def run_ours(args):
     assert int(status.item()) == 0, f"kernel status {status.item()}"
     del g_step, g_dec
 
-    if dist is not None:
-        t = torch.tensor([elapsed_ms, e2e_ms, dec_avg_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms, dec_avg_ms = t.tolist()
+    elapsed_ms, e2e_ms, dec_avg_ms = max_over_ranks(dist, [elapsed_ms, e2e_ms, dec_avg_ms], "cuda")
 
     ms_per_step = elapsed_ms / args.steps
     kv_bytes_step = kv_bytes_layer * L
-    value = world * kv_bytes_step / (ms_per_step * 1e-3) / 1e9
-    e2e_value = world * kv_bytes_step / (e2e_ms / args.steps * 1e-3) / 1e9
+    value = weak_scaling_gbs(world, kv_bytes_step, ms_per_step)
+    e2e_value = weak_scaling_gbs(world, kv_bytes_step, e2e_ms / args.steps)
     tok_s = world * w.batch / (ms_per_step * 1e-3)
     peak, peak_kind = peaks()
     achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
