@@ -46,9 +46,15 @@ def peaks():
 
 
 def decode_source_hash() -> str:
+    """Hash of the decode kernel's code (comments and whitespace removed), the
+    key under which profiles/decode_traffic.json records ncu DRAM counters."""
+    import re
     h = hashlib.sha256()
     for f in ("kvq_decode.cu", "kvq_internal.cuh"):
-        h.update(open(os.path.join(ROOT, "quantized_kv_cache_17_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "quantized_kv_cache_17_b200", "csrc", f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,7 +1,8 @@
 // paged_decode_attn_{int8,q4_0,k8v4}: split-K single-token attention over the
 // quantised, paged KV cache, one CTA per work unit of the plan; attn_combine:
 // the merge of a (sequence, KV head) group's partials, either as its own
-// launch or fused into the last CTA of the group.
+// launch or fused into the decode (all CTAs of the group merging one head each
+// under a cooperative launch, else the group's last CTA).
 //
 // [Strata] "4-bit KV 缓存：先旋转，再压到 4-bit": scores are taken on the rotated
 // query and rotated keys (<Hq, Hk> = <q, k>), values are mixed in the rotated
@@ -13,16 +14,17 @@
 // steps (8 tiles, contiguous inside one page block) with 1-D bulk copies into
 // a ring of shared-memory stages guarded by full/empty mbarriers.  At the end
 // the CTA merges its warps' softmax states in shared memory and writes one
-// partial (o[G][256] unnormalised, m[8], l[8]; scores in log2 units); with the
-// combine fused in, the last CTA of each (sequence, KV head) merges the group.
+// partial (o[G][256] unnormalised, m[8], l[8]; scores in log2 units), then,
+// with the combine fused in, takes part in the merge of its group.
 //
 // Tensor-core kernel (the product), warp-specialised:
 //  - QK warps: the query of the group as mma.sync m16n8k16 A fragments in
 //    registers (rows = [8 heads, fp16 hi | same 8 heads, fp16 lo], k = 16
-//    dims), K codes unpacked to fp16 in registers as B (cols = 8 tokens),
-//    the per-block K scale applied to the fp32 block sums; online softmax;
-//    hands p (and the rescale factor of each head) to its PV warp through a
-//    small shared-memory ring.
+//    dims), K codes as stored placed in fp16 words as B (cols = 8 tokens;
+//    exact subnormals, the code offset removed by one m16n8k8 per tile), the
+//    per-block K scale applied to the fp32 block sums; online softmax; hands
+//    p (and the rescale factor of each head) to its PV warp through a 2-slot
+//    shared-memory ring.
 //  - PV warps: the output accumulators o[dims][heads] in registers; rows = 16
 //    dims of V codes (exact in fp16), k = [8 tokens with P'hi | the same 8
 //    tokens with P'lo], P' = p * dV formed as an exact fp16 pair.  The score
