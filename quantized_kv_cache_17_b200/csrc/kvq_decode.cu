@@ -146,6 +146,11 @@ template <int FMT> struct TcCfg {
     // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]
     static constexpr int TOTAL = BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 16;
     static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+    // A QK warp waits on the ready barrier of the stage of its next item, which
+    // lies (NQK items later) at most this many stages ahead of its last one; a
+    // wait more than one lap of the ring ahead of the barrier's pending phase
+    // would be satisfied by an older phase of the same parity.
+    static_assert((NQK + ITEMS_PER_STAGE - 1) / ITEMS_PER_STAGE < NS, "QK item stride must stay within one ring lap");
 };
 
 // Scores are formed from the codes as stored (q4_0 nibbles 0..15, int8 codes
