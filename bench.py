@@ -50,7 +50,7 @@ def decode_source_hash() -> str:
     key under which profiles/decode_traffic.json records ncu DRAM counters."""
     import re
     h = hashlib.sha256()
-    for f in ("kvq_decode.cu", "kvq_internal.cuh"):
+    for f in ("kvq_decode.cu", "kvq_internal.cuh", "kvq_append_dev.cuh"):
         text = open(os.path.join(ROOT, "quantized_kv_cache_17_b200", "csrc", f)).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
@@ -245,6 +245,10 @@ def run_ours(args):
     kv_bytes_layer = sum(w.seq_lens) * w.n_kv_heads * layout.bytes_per_token_head
 
     def layer_step(l):
+        if fused:       # kv_append, q_rotate and the decode with its merge: one launch
+            kvq.paged_decode_step(dw.pool, l, q[l], k_new[l], v_new[l], dw.page_table, plan_d, info, ws, out_bf[l],
+                                  out_f[l], status)
+            return
         qq = q[l]
         if rot_q:       # q_rotate and kv_append in one launch
             kvq.kv_append_q_rotate(dw.pool, l, k_new[l], v_new[l], pos, dw.page_table, qq, q_rot[l], status=status)
@@ -271,7 +275,7 @@ def run_ours(args):
             else:
                 kvq.paged_decode_attn(dw.pool, l, qq, dw.page_table, plan_d, info, ws, status, cudacore=use_alu)
 
-    launches_per_layer = 2 if fused else 3      # (kv_append[_q_rotate], decode[, combine])
+    launches_per_layer = 1 if fused else 3      # paged_decode_step, or (kv_append[_q_rotate], decode, combine)
 
     def barrier():
         if dist is not None:
@@ -279,6 +283,8 @@ def run_ours(args):
 
     # eager warm-up (sets kernel attributes, fills caches of the runtime), then
     # capture one whole step and the decode launches alone as CUDA graphs
+    if rot_q:
+        kvq.q_rotate(q, q_rot)      # the decode-only graph takes the rotated query
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -363,8 +369,16 @@ def run_ours(args):
     e2e_value = weak_scaling_gbs(world, kv_bytes_step, e2e_ms / args.steps)
     tok_s = world * w.batch / (ms_per_step * 1e-3)
     peak, peak_kind = peaks()
-    achieved = kv_bytes_layer / (dec_avg_ms * 1e-3) / 1e9
-    kernel_tag = "decode_alu" if use_alu else ("decode_mma_fused" if fused else "decode_mma")
+    if fused:
+        # the timed region runs the decode step kernel alone, once per layer:
+        # its average launch is the region's time over its launches
+        launch_ms = ms_per_step / L
+        kernel_tag = "decode_step_fused"
+    else:
+        # several kernels per layer: the decode is timed on its own graph
+        launch_ms = dec_avg_ms
+        kernel_tag = "decode_alu" if use_alu else "decode_mma"
+    achieved = kv_bytes_layer / (launch_ms * 1e-3) / 1e9
     traffic = ncu_traffic(kernel_tag, w.name)
 
     cpu = None
@@ -406,6 +420,7 @@ def run_ours(args):
                              "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                              if peak_kind == "measured" else "fallback 6.65 TB/s",
                              "bytes_per_launch": kv_bytes_layer,
+                             "us_per_launch": round(launch_ms * 1e3, 3),
                              "kernel": kernel_tag},
                 "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},

@@ -227,6 +227,35 @@ int paged_decode_attn_k8v4_combined(const kvq_pool *pool, int layer, const float
                                     uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
                                     void *stream);
 
+/* paged_decode_step_<fmt>: one whole decode step of one layer in a single
+ * launch: kv_append of every sequence's newest token, q_rotate of the raw
+ * query (q4_0; int8 and k8v4 take the query as it is) and
+ * paged_decode_attn_<fmt>_combined over the updated cache.  The results, pool
+ * bytes and outputs, are bit-identical to those three calls.
+ *  q         device fp32 [n_seq][n_q_heads][256], the raw query
+ *  k_new, v_new device fp32 [n_seq][n_kv_heads][256]: the token at position
+ *            seq_len - 1 of each sequence (seq_len as given to kvq_decode_plan)
+ * The CTA whose unit ends each (sequence, KV head) range encodes that range's
+ * token into the pool at its start, and writes the same codes into its copy of
+ * the token's tile when the tile lands in shared memory (the copy may predate
+ * the pool write); the pool bytes of the tile's other tokens are untouched.  A
+ * page slot out of range sets KVQ_STATUS_BAD_SLOT as in kv_append.  Other
+ * arguments, contract and errors as paged_decode_attn_<fmt>_combined.  The
+ * pages describe the three steps separately; this entry only merges their
+ * launches. */
+int paged_decode_step_int8(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,
+                           const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
+                           float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
+                           int32_t *status, void *stream);
+int paged_decode_step_q4_0(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,
+                           const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
+                           float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
+                           int32_t *status, void *stream);
+int paged_decode_step_k8v4(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,
+                           const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
+                           float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
+                           int32_t *status, void *stream);
+
 /* paged_decode_attn_q4_0_noalloc: paged_decode_attn_q4_0_combined without a
  * workspace argument, for callers that cannot allocate device memory.  Some
  * hosts own all device memory and pass a library only the buffers of the call

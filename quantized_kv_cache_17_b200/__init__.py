@@ -35,7 +35,8 @@ EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_a
            "kvq_decode_plan",
            "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
            "paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined", "paged_decode_attn_k8v4_combined",
-           "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine"]
+           "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine",
+           "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4"]
 
 
 class KVQError(RuntimeError):
@@ -90,6 +91,10 @@ def lib():
             getattr(L, n).argtypes = dec[:-2] + [P, P] + dec[-2:]
         L.paged_decode_attn_q4_0_noalloc.argtypes = dec[:7] + [P, P, P, P]
         L.paged_decode_attn_cudacore.argtypes = [I32] + dec
+        for n in ("paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4"):
+            getattr(L, n).argtypes = [ctypes.POINTER(Pool), I32, P, P, P, P, I32, P, ctypes.POINTER(PlanInfo), P,
+                                      ctypes.c_uint64,
+                                      P, P, P, P]
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
         for n in EXPORTS[1:]:
             getattr(L, n).restype = ctypes.c_int
@@ -218,6 +223,22 @@ def paged_decode_attn_combined(pool: KVPool, layer: int, q, page_table, plan_dev
     name = _DECODE[pool.fmt] + "_combined"
     _check(getattr(lib(), name)(ctypes.byref(cp), layer, _ptr(q), _ptr(page_table), page_table.shape[1],
                                 _ptr(plan_dev), ctypes.byref(info), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _ptr(out_bf16), _ptr(out_f32),
+                                _ptr(status), _stream(stream)), name)
+
+
+_STEP = {INT8: "paged_decode_step_int8", Q4_0: "paged_decode_step_q4_0", K8V4: "paged_decode_step_k8v4"}
+
+
+def paged_decode_step(pool: KVPool, layer: int, q, k_new, v_new, page_table, plan_dev, info: PlanInfo, workspace,
+                      out_bf16, out_f32=None, status=None, stream=None):
+    """One decode step of a layer in one launch: append every sequence's newest
+    token (k_new, v_new [n_seq, n_kv_heads, 256] at position seq_len - 1),
+    rotate the raw query q where the format does, decode and merge."""
+    cp = pool.c_pool()
+    name = _STEP[pool.fmt]
+    _check(getattr(lib(), name)(ctypes.byref(cp), layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(page_table),
+                                page_table.shape[1], _ptr(plan_dev), ctypes.byref(info), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _ptr(out_bf16), _ptr(out_f32),
                                 _ptr(status), _stream(stream)), name)
 

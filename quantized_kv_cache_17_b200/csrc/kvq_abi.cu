@@ -63,7 +63,7 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ECUDA; }
 int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                   int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                   uint64_t workspace_bytes, int32_t *status, void *stream, uint16_t *out_bf16 = nullptr,
-                  float *out_f32 = nullptr) {
+                  float *out_f32 = nullptr, const float *k_new = nullptr, const float *v_new = nullptr) {
     PoolGeom geo;
     int rc = check_pool(pool, layer, &geo);
     if (rc) return rc;
@@ -80,7 +80,7 @@ int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float
     const int inverse = fmt == KVQ_INT8 ? 0 : 1;
     return cuda_rc(launch_decode(fmt, tc, static_cast<const uint8_t *>(pool->base), geo, layer, q, page_table,
                                  max_pages, plan, *info, workspace, status, inverse, out_bf16, out_f32,
-                                 static_cast<cudaStream_t>(stream)));
+                                 static_cast<cudaStream_t>(stream), k_new, v_new));
 }
 
 }  // namespace
@@ -268,6 +268,21 @@ KVQ_COMBINED(paged_decode_attn_int8_combined, KVQ_INT8)
 KVQ_COMBINED(paged_decode_attn_q4_0_combined, KVQ_Q4_0)
 KVQ_COMBINED(paged_decode_attn_k8v4_combined, KVQ_K8V4)
 #undef KVQ_COMBINED
+
+#define KVQ_STEP(NAME, FMT)                                                                                     \
+    int NAME(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,              \
+             const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,            \
+             float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,      \
+             void *stream) {                                                                                       \
+        if (!out_bf16 || !k_new || !v_new) return KVQ_EINVAL;                                                      \
+        if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_EALIGN;                                             \
+        return decode_common(FMT, true, pool, layer, q, page_table, max_pages, plan, info, workspace,             \
+                             workspace_bytes, status, stream, out_bf16, out_f32, k_new, v_new);                   \
+    }
+KVQ_STEP(paged_decode_step_int8, KVQ_INT8)
+KVQ_STEP(paged_decode_step_q4_0, KVQ_Q4_0)
+KVQ_STEP(paged_decode_step_k8v4, KVQ_K8V4)
+#undef KVQ_STEP
 
 int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,
                  uint16_t *out_bf16, float *out_f32, void *stream) {

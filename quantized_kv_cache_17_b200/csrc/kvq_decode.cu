@@ -35,6 +35,7 @@
 #include <type_traits>
 
 #include "kvq_internal.cuh"
+#include "kvq_append_dev.cuh"
 
 namespace kvq {
 namespace {
@@ -143,8 +144,11 @@ template <int FMT> struct TcCfg {
     static constexpr int SFOFF = (DATA + 127) & ~127;
     static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
     static constexpr int BAR_OFF = POFF + NQK * DP * PSLOT * 4;
-    // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]
-    static constexpr int TOTAL = BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 16;
+    static_assert(!Fmt<FMT>::KROT || NQK * DP * PSLOT >= 8 * D, "the hand-over ring holds the rotated query of a decode step");
+    // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]; then,
+    // for a decode step, the newest token's codes and scales (5 words per lane)
+    static constexpr int TKV_OFF = (BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 15) & ~15;
+    static constexpr int TOTAL = TKV_OFF + 32 * 5 * 4;
     static_assert(TOTAL <= 227 * 1024, "shared memory budget");
     // A QK warp waits on the ready barrier of the stage of its next item, which
     // lies (NQK items later) at most this many stages ahead of its last one; a
@@ -1001,6 +1005,12 @@ struct DecodeArgs {
     uint16_t *out_bf16;    // fused combine outputs (NULL: write partials only)
     float *out_f32;
     int coop;              // fused combine: every CTA is resident (cooperative launch); merge heads in parallel
+    // decode step (tensor-core kernel only): q is the raw query, rotated in the
+    // kernel where the format rotates; k_new / v_new [n_seq][n_kv][256] are the
+    // sequences' newest tokens (position seq_len - 1), appended by the last
+    // CTA of each (sequence, KV head) group before it fetches that position
+    const float *k_new;
+    const float *v_new;
 };
 
 // ---------------------------------------------------------------------------
@@ -1027,9 +1037,13 @@ __device__ __forceinline__ bool unit_ok(const DecodeArgs &A, int seq, int kvh, i
 // lanes fetch the page slots of 32 pages at a time (one load round trip per 32
 // pages instead of one per step); lane 0 waits for free stages and issues the
 // bulk copies.
-template <int NS, int STAGE_BYTES, int TILE_BYTES>
+struct NoHook {
+    __device__ __forceinline__ void operator()(int, int) const {}
+};
+template <int NS, int STAGE_BYTES, int TILE_BYTES, class Hook = NoHook>
 __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, uint64_t *full, uint64_t *empty,
-                                          int *stage_ok, int seq, int kvh, int t0, int n_steps, int lane) {
+                                          int *stage_ok, int seq, int kvh, int t0, int n_steps, int lane,
+                                          Hook hook = Hook()) {
     const uint8_t *head_base = A.pool + (int64_t)A.layer * A.geo.layer_stride + (int64_t)kvh * A.geo.page_bytes;
     const int32_t *pt = A.page_table + (int64_t)seq * A.max_pages;
     const uint64_t pol = policy_evict_first();
@@ -1045,6 +1059,7 @@ __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, ui
             my_slot = pg < A.max_pages ? __ldg(pt + pg) : -1;
         }
         const int slot = __shfl_sync(0xffffffffu, my_slot, rel & 31);
+        hook(i, lane);                 // whole warp, before step i is requested
         if (lane == 0 && !stop) {
             const int si = i % NS;
             if (i >= NS && !mbar_wait_bounded(&empty[si], ((i / NS) - 1) & 1, WAIT_LIMIT_NS)) {
@@ -1135,11 +1150,80 @@ __device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_
     publish_unit<FUSED, NCT>(A, seq, kvh, n_units, s_last, smem);
 }
 
+// Decode step helpers, kept out of line so that their registers do not shape
+// the allocation of the kernel's main loop.  In the CTA whose unit ends the
+// group, the scale warp encodes the newest token into the pool while the first
+// stages land, and keeps its codes in shared memory, to write them into the
+// last stage when it lands.
+// The QK warps rotate the raw query heads h = first, first + stride, ... into
+// q_s.
+// Encode the newest token into the pool and keep its codes and scales in
+// shared memory (5 words per lane).
+template <int FMT>
+__device__ __noinline__ void step_encode_token(const DecodeArgs &A, int seq, int kvh, int pos, uint32_t *stash,
+                                               int lane) {
+    const int64_t row = ((int64_t)seq * A.geo.n_kv_heads + kvh) * D;
+    float xk[8], xv[8];
+    load8(A.k_new + row + lane * 8, xk);
+    load8(A.v_new + row + lane * 8, xv);
+    const bool in_range = pos >= 0 && pos < A.max_pages * PAGE;
+    const int slot = in_range ? A.page_table[(int64_t)seq * A.max_pages + (pos >> 8)] : -1;
+    TokenCodes t;
+    quant_token<FMT>(xk, xv, lane, t);
+    uint8_t *gtile = token_tile<FMT>(const_cast<uint8_t *>(A.pool), A.geo, A.layer, slot, kvh, pos, A.status, lane);
+    if (gtile) store_token<FMT>(t, lane, pos & 7, gtile);
+    uint32_t w[5];
+    w[4] = (uint32_t)__half_as_ushort(t.dk) | ((uint32_t)__half_as_ushort(t.dv) << 16);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        w[h] = w[2 + h] = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            w[h] |= (uint32_t)(t.k[4 * h + e] & 0xFF) << (8 * e);
+            w[2 + h] |= (uint32_t)(t.v[4 * h + e] & 0xFF) << (8 * e);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 5; ++i) stash[lane * 5 + i] = w[i];
+    __syncwarp();
+}
+// Write the stashed token into the landed stage that holds it, over the bytes
+// the copy brought (which may predate the pool store above).
+template <int FMT>
+__device__ __noinline__ void step_patch_stage(int pos, const uint32_t *stash, uint8_t *stage, int lane) {
+    TokenCodes t;
+    uint32_t w[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = stash[lane * 5 + i];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            t.k[4 * h + e] = (w[h] >> (8 * e)) & 0xFF;
+            t.v[4 * h + e] = (w[2 + h] >> (8 * e)) & 0xFF;
+        }
+    t.dk = __ushort_as_half((unsigned short)(w[4] & 0xFFFF));
+    t.dv = __ushort_as_half((unsigned short)(w[4] >> 16));
+    store_token<FMT>(t, lane, pos & 7, stage + ((pos & 63) >> 3) * TileLayout<FMT>::BYTES);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // before the stage's next bulk fill
+    __syncwarp();
+}
+__device__ __noinline__ void step_rotate_query(const float *qg, float *q_s, int G, int first, int stride, int lane) {
+    for (int h = first; h < G; h += stride) {
+        float x[8];
+        load8(qg + h * D + lane * 8, x);
+        fwht256_lane(x, lane);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q_s[h * D + lane * 8 + i] = x[i];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core kernel
 // ---------------------------------------------------------------------------
-template <int FMT, bool FUSED>
-__global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(const DecodeArgs A) {
+template <int FMT, bool FUSED, bool STEP = false>
+__global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(const __grid_constant__ DecodeArgs A) {
+    static_assert(!STEP || FUSED, "the decode step merges in the kernel");
     using L = TileLayout<FMT>;
     using C = TcCfg<FMT>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -1176,18 +1260,24 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         fence_mbar_init();
     }
     __syncthreads();
+    // decode step: the last CTA of the group appends the group's newest token
+    const bool appends = STEP && u == A.plan[PLAN_HEADER + 4 * n_units + seq * A.geo.n_kv_heads + kvh + 1] - 1;
 
     if (warp == C::COPY_WARP) {
         copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
         return;
     }
     if (warp == C::SCALE_WARP) {
+        uint32_t *stash = reinterpret_cast<uint32_t *>(smem + C::TKV_OFF);
+        if (appends) step_encode_token<FMT>(A, seq, kvh, t1 - 1, stash, lane);
         for (int i = 0; i < n_steps; ++i) {
             const int si = i % C::NS;
             if (!mbar_wait_bounded(&full[si], (i / C::NS) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
+            if (appends && i == n_steps - 1 && stage_ok[si])    // the stage that holds the newest token
+                step_patch_stage<FMT>(t1 - 1, stash, smem + si * C::STAGE_BYTES, lane);
             if (stage_ok[si])
                 convert_stage_scales<FMT>(smem + si * C::STAGE_BYTES,
                                           reinterpret_cast<float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES), lane);
@@ -1208,7 +1298,16 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     // to its PV warp with the scores.  (Handing items out from a shared counter
     // instead measured slower on long units.)
     if (is_qk) {
-        qk.init(A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D, G, lane);
+        const float *qg = A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D;
+        if constexpr (STEP && Fmt<FMT>::KROT) {
+            // decode step: rotate the group's raw query into the (still unused)
+            // hand-over ring, exactly as q_rotate would; head h by QK warp h % NQK
+            step_rotate_query(qg, pring, G, pw, C::NQK, lane);
+            asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+            qg = pring;
+        }
+        qk.init(qg, G, lane);
+        if constexpr (STEP && Fmt<FMT>::KROT) asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
         for (int k = 0;; ++k) {
             const int slot = k % C::DP;
             float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
@@ -1467,6 +1566,13 @@ cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s
             if (cap[dev] == 0) cap[dev] = resident_ctas(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS);
             b.coop = n_units <= cap[dev] && n_units <= MH_MAX_UNITS ? 1 : 0;
         }
+        if constexpr (FUSED) {
+            if (b.k_new) {
+                static bool cfg_step = false;
+                return launch_k(decode_tc_kernel<FMT, true, true>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS, b, n_units, s,
+                                cfg_step);
+            }
+        }
         return launch_k(decode_tc_kernel<FMT, FUSED>, TcCfg<FMT>::TOTAL, TcCfg<FMT>::NTHREADS, b, n_units, s, cfg);
     }
     static bool c4 = false, c6 = false, c8 = false;
@@ -1491,9 +1597,9 @@ cudaError_t launch_fused(int fmt, bool tc, const DecodeArgs &a, int n_units, cud
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
                           const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht, uint16_t *out_bf16,
-                          float *out_f32, cudaStream_t s) {
+                          float *out_f32, cudaStream_t s, const float *k_new, const float *v_new) {
     DecodeArgs a{pool, geo, layer, q, page_table, max_pages, plan, info.n_kv_heads * info.group, info.group, ws,
-                 status, inverse_fwht, out_bf16, out_f32, 0};
+                 status, inverse_fwht, out_bf16, out_f32, 0, k_new, v_new};
     if (out_bf16) return launch_fused<true>(fmt, tensor_cores, a, info.n_units, s);
     return launch_fused<false>(fmt, tensor_cores, a, info.n_units, s);
 }

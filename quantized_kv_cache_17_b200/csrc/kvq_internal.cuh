@@ -280,7 +280,8 @@ cudaError_t launch_append_rotate(int fmt, uint8_t *pool, const PoolGeom &geo, in
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
                           const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht,
-                          uint16_t *out_bf16, float *out_f32, cudaStream_t s);
+                          uint16_t *out_bf16, float *out_f32, cudaStream_t s, const float *k_new = nullptr,
+                          const float *v_new = nullptr);
 cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_info &info, int inverse_fwht,
                            uint16_t *out_bf16, float *out_f32, cudaStream_t s);
 

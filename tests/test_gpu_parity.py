@@ -211,3 +211,43 @@ def test_kv_append_q_rotate_matches_separate_calls(fmt):
     qc = kvq.kv_append_q_rotate(b.pool, 0, None, None, pos, b.page_table, q[0])    # rotation only
     torch.cuda.synchronize()
     assert torch.equal(qc.view(torch.int32), qa.view(torch.int32))
+
+
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("case", ["ragged_g6", "ragged_g8", "cross_page_1025"])
+def test_decode_step_matches_the_three_calls(case, fmt):
+    """paged_decode_step = kv_append of the newest tokens + q_rotate + the
+    combined decode: the same pool bytes and the same output bits, and the
+    output within the tolerance of the oracle."""
+    w, _ = _case(case, fmt)
+    a = kdev.build_pool(w, extra_slots=2, prefill_last=False)
+    b = kdev.build_pool(w, extra_slots=2, prefill_last=False)
+    q, k, v, pos = kdev.step_inputs(w, [0])
+    # stale bytes in the new token's row, which the step's copy of that tile may read
+    for dw in (a, b):
+        kvq.kv_append(dw.pool, 0, (-2.0 * k[0]).contiguous(), (0.5 * v[0].flip(-1)).contiguous(), pos, dw.page_table)
+    plan, info = kvq.decode_plan(a.pool.desc, a.seq_lens, a.page_table.shape[1], 0)
+    plan_d = torch.from_numpy(plan).cuda()
+    outs = []
+    for dw, fused_step in ((a, False), (b, True)):
+        ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out_bf = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+        out_f = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
+        if fused_step:
+            kvq.paged_decode_step(dw.pool, 0, q[0], k[0], v[0], dw.page_table, plan_d, info, ws, out_bf, out_f, status)
+        else:
+            kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table, status=status)
+            qp = kvq.q_rotate(q[0]) if kvq.rotated_q(fmt) else q[0]
+            kvq.paged_decode_attn_combined(dw.pool, 0, qp, dw.page_table, plan_d, info, ws, out_bf, out_f, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        outs.append((out_f.cpu(), out_bf.cpu()))
+    assert torch.equal(a.pool.buf, b.pool.buf)
+    assert torch.equal(outs[0][0].view(torch.int32), outs[1][0].view(torch.int32))
+    assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
+    G = w.group
+    got = outs[1][0].numpy()
+    for bb in range(w.batch):
+        for g in range(w.n_kv_heads):
+            gc.assert_close(got[bb, g * G:(g + 1) * G], gc.oracle_group(b, 0, bb, g), f"step/{case}/{fmt}")
