@@ -1150,13 +1150,12 @@ __device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_
     publish_unit<FUSED, NCT>(A, seq, kvh, n_units, s_last, smem);
 }
 
-// Decode step helpers, kept out of line so that their registers do not shape
-// the allocation of the kernel's main loop.  In the CTA whose unit ends the
+// Helpers kept out of line so that their registers do not shape the allocation
+// of the kernel's main loop.  In a decode step, in the CTA whose unit ends the
 // group, the scale warp encodes the newest token into the pool while the first
 // stages land, and keeps its codes in shared memory, to write them into the
-// last stage when it lands.
-// The QK warps rotate the raw query heads h = first, first + stride, ... into
-// q_s.
+// last stage when it lands.  The QK warps copy the query heads h = first,
+// first + stride, ... into q_s, rotating them (ROTATE) in a decode step.
 // Encode the newest token into the pool and keep its codes and scales in
 // shared memory (5 words per lane).
 template <int FMT>
@@ -1208,11 +1207,12 @@ __device__ __noinline__ void step_patch_stage(int pos, const uint32_t *stash, ui
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // before the stage's next bulk fill
     __syncwarp();
 }
-__device__ __noinline__ void step_rotate_query(const float *qg, float *q_s, int G, int first, int stride, int lane) {
+template <bool ROTATE>
+__device__ __noinline__ void step_stage_query(const float *qg, float *q_s, int G, int first, int stride, int lane) {
     for (int h = first; h < G; h += stride) {
         float x[8];
         load8(qg + h * D + lane * 8, x);
-        fwht256_lane(x, lane);
+        if (ROTATE) fwht256_lane(x, lane);
 #pragma unroll
         for (int i = 0; i < 8; ++i) q_s[h * D + lane * 8 + i] = x[i];
     }
@@ -1299,15 +1299,21 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     // instead measured slower on long units.)
     if (is_qk) {
         const float *qg = A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D;
-        if constexpr (STEP && Fmt<FMT>::KROT) {
-            // decode step: rotate the group's raw query into the (still unused)
-            // hand-over ring, exactly as q_rotate would; head h by QK warp h % NQK
-            step_rotate_query(qg, pring, G, pw, C::NQK, lane);
+        // The group's query goes through the (still unused) hand-over ring, one
+        // head per QK warp, where the ring holds the largest group: a warp that
+        // loads all G heads itself waits longer while the first stages flood
+        // the memory system.  A decode step rotates the raw query on the way,
+        // as q_rotate would.  (The int8 ring holds 7 heads; choosing at run time
+        // by G measured slower for every format.)
+        constexpr bool ROT = STEP && Fmt<FMT>::KROT;
+        constexpr bool QSTAGE = C::NQK * C::DP * C::PSLOT >= KVQ_MAX_GROUP * D;
+        if constexpr (QSTAGE) {
+            step_stage_query<ROT>(qg, pring, G, pw, C::NQK, lane);
             asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
             qg = pring;
         }
         qk.init(qg, G, lane);
-        if constexpr (STEP && Fmt<FMT>::KROT) asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+        if constexpr (QSTAGE) asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
         for (int k = 0;; ++k) {
             const int slot = k % C::DP;
             float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
