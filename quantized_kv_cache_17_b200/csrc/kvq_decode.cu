@@ -143,8 +143,9 @@ template <int FMT> struct TcCfg {
     static constexpr int DATA = RING > MERGE ? RING : MERGE;
     static constexpr int SFOFF = (DATA + 127) & ~127;
     static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
-    static constexpr int BAR_OFF = POFF + NQK * DP * PSLOT * 4;
-    static_assert(!Fmt<FMT>::KROT || NQK * DP * PSLOT >= 8 * D, "the hand-over ring holds the rotated query of a decode step");
+    // the QK -> PV rings; before the loop, the group's query (KVQ_MAX_GROUP heads)
+    static constexpr int PRING_FLOATS = NQK * DP * PSLOT > KVQ_MAX_GROUP * D ? NQK * DP * PSLOT : KVQ_MAX_GROUP * D;
+    static constexpr int BAR_OFF = POFF + PRING_FLOATS * 4;
     // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]; then,
     // for a decode step, the newest token's codes and scales (5 words per lane)
     static constexpr int TKV_OFF = (BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 15) & ~15;
@@ -1300,20 +1301,13 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     if (is_qk) {
         const float *qg = A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D;
         // The group's query goes through the (still unused) hand-over ring, one
-        // head per QK warp, where the ring holds the largest group: a warp that
-        // loads all G heads itself waits longer while the first stages flood
-        // the memory system.  A decode step rotates the raw query on the way,
-        // as q_rotate would.  (The int8 ring holds 7 heads; choosing at run time
-        // by G measured slower for every format.)
-        constexpr bool ROT = STEP && Fmt<FMT>::KROT;
-        constexpr bool QSTAGE = C::NQK * C::DP * C::PSLOT >= KVQ_MAX_GROUP * D;
-        if constexpr (QSTAGE) {
-            step_stage_query<ROT>(qg, pring, G, pw, C::NQK, lane);
-            asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
-            qg = pring;
-        }
-        qk.init(qg, G, lane);
-        if constexpr (QSTAGE) asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+        // head per QK warp: a warp that loads all G heads itself waits longer
+        // while the first stages flood the memory system.  A decode step
+        // rotates the raw query on the way, as q_rotate would.
+        step_stage_query<STEP && Fmt<FMT>::KROT>(qg, pring, G, pw, C::NQK, lane);
+        asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+        qk.init(pring, G, lane);
+        asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
         for (int k = 0;; ++k) {
             const int slot = k % C::DP;
             float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
