@@ -13,15 +13,17 @@ REL_L2 = 1e-3     # attention output tolerance, fp32 output vs fp64 oracle
 MAX_ABS = 2e-3
 
 
-def decode_step(dw, layer, q, impl="mma", n_ctas=0, status=None, mode="split", repeat=1):
+def decode_step(dw, layer, q, impl="mma", n_ctas=0, status=None, mode="split", repeat=1, k_new=None, v_new=None):
     """q: [B, Hq, 256] fp32 device (unrotated).  mode 'split': decode then
     attn_combine; 'fused': the *_combined entry point (run `repeat` times on the
-    same workspace).  Returns (out_f32, out_bf16, status, plan, info)."""
+    same workspace); 'step': paged_decode_step, which also appends k_new / v_new
+    ([B, Hkv, 256], the token at seq_len - 1) and rotates q itself.
+    Returns (out_f32, out_bf16, status, plan, info)."""
     w = dw.w
     plan, info = kvq.decode_plan(dw.pool.desc, dw.seq_lens, dw.page_table.shape[1], n_ctas)
     plan_d = torch.from_numpy(plan).cuda()
     ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
-    qp = kvq.q_rotate(q) if kvq.rotated_q(w.fmt) else q
+    qp = kvq.q_rotate(q) if kvq.rotated_q(w.fmt) and mode != "step" else q
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out_bf = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
@@ -29,7 +31,10 @@ def decode_step(dw, layer, q, impl="mma", n_ctas=0, status=None, mode="split", r
     for _ in range(repeat):
         out_bf.fill_(float("nan"))
         out_f.fill_(float("nan"))
-        if mode == "fused":
+        if mode == "step":
+            kvq.paged_decode_step(dw.pool, layer, q, k_new, v_new, dw.page_table, plan_d, info, ws, out_bf, out_f,
+                                  status)
+        elif mode == "fused":
             kvq.paged_decode_attn_combined(dw.pool, layer, qp, dw.page_table, plan_d, info, ws, out_bf, out_f, status)
         else:
             kvq.paged_decode_attn(dw.pool, layer, qp, dw.page_table, plan_d, info, ws, status,

@@ -1,5 +1,5 @@
 """Parity at the full workload sizes, in the launch configuration the benchmark
-times (plan with one unit per SM, the tensor-core kernels), on sampled
+times (plan with one unit per SM, the decode step kernel), on sampled
 outputs the oracle computes one at a time: whole (sequence, KV head) groups of
 attention output over the full context, and bit-exact codes for sampled token
 positions regenerated on the CPU."""
@@ -32,15 +32,20 @@ def built():
         pytest.skip("no CUDA device")
 
 
+@pytest.mark.parametrize("mode", ["step", "fused"])
 @pytest.mark.parametrize("name", list(SAMPLES))
-def test_full_size_sampled(name):
+def test_full_size_sampled(name, mode):
+    """mode 'step': paged_decode_step, the launch the benchmark times (it
+    appends the newest token itself); 'fused': kv_append, then the combined
+    decode."""
     w = kvq_inputs.workload(name)
     layer = w.n_layers - 1
     dw = kdev.build_pool(w, layers=[layer], extra_slots=7)
     q, k, v, pos = kdev.step_inputs(w, [layer])
     import quantized_kv_cache_17_b200 as kvq
-    kvq.kv_append(dw.pool, layer, k[0], v[0], pos, dw.page_table)
-    out_f, out_bf, status, plan, info = gc.decode_step(dw, layer, q[0], mode="fused")
+    if mode == "fused":
+        kvq.kv_append(dw.pool, layer, k[0], v[0], pos, dw.page_table)
+    out_f, out_bf, status, plan, info = gc.decode_step(dw, layer, q[0], mode=mode, k_new=k[0], v_new=v[0])
     assert status == 0
     rng = np.random.default_rng(w.seed)
     G = w.group
