@@ -783,11 +783,15 @@ __device__ __forceinline__ void finish_row(float (&x)[8], int lane, int inverse_
 // o = sum 2^(m_u - M) o_u / L, then H/16 if V was stored rotated.  Runs on the
 // first NTH threads of the CTA (named barrier bar_id); sm: COMBINE_SMEM floats.
 // Warp h computes head h's weights from all units' (m, l) at once (warp max
-// and sum); then every lane keeps 2 UB independent 16-byte loads in flight.
+// and sum); then every lane keeps 2 UB independent 16-byte loads in flight,
+// and the warps that share a head add their sums in a fixed order.  Out of
+// line, so that it does not shape the register allocation of the decode's
+// main loop.
 // ---------------------------------------------------------------------------
 template <int NTH>
-__device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t out_row, int inverse_fwht,
-                              uint16_t *out_bf16, float *out_f32, float *sm, int bar_id) {
+__device__ __noinline__ void combine_group(const float *ws, int G, int u0, int u1, int64_t out_row,
+                                           int inverse_fwht, uint16_t *out_bf16, float *out_f32, float *sm,
+                                           int bar_id) {
     constexpr int NWARP = NTH / 32;
     static_assert(NWARP >= 8, "the weight pass takes one warp per head");
     constexpr int UB = 8;                         // units whose loads are in flight together (16 float4 / lane)
@@ -844,9 +848,9 @@ __device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t ou
         // warps per head: warp w takes head w % G and every wph-th unit, UB units
         // (2 UB independent 16-byte loads per lane) at a time
         const int wph = NWARP / G;
+        const int h = warp % G, part = warp / G;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         if (warp < wph * G) {
-            const int h = warp % G, part = warp / G;
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             for (int ub = part; ub < n; ub += UB * wph) {
                 float4 a[UB], b[UB];
 #pragma unroll
@@ -867,15 +871,16 @@ __device__ void combine_group(const float *ws, int G, int u0, int u1, int64_t ou
                     acc[6] = fmaf(b[j].z, f, acc[6]); acc[7] = fmaf(b[j].w, f, acc[7]);
                 }
             }
-            if (wph == 1) {
+        }
+        // the parts of a head add their sums in part order, so that the result
+        // does not depend on which warp finishes first
+        for (int p = 0; p < wph; ++p) {
+            if (warp < wph * G && part == p) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) o_s[h * D + lane * 8 + i] += acc[i];
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) atomicAdd(o_s + h * D + lane * 8 + i, acc[i]);
             }
+            asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
         }
-        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NTH));
     }
     // warp h finishes head h
     for (int h = warp; h < G; h += NWARP) {

@@ -193,6 +193,23 @@ def test_decode_bad_plan_reports_status():
     assert int(status.item()) & kvq.STATUS_BAD_PLAN
 
 
+@pytest.mark.parametrize("mode", ["split", "fused"])
+@pytest.mark.parametrize("G,n_ctas", [(4, 300), (6, 300), (4, 0)])
+def test_group_merge_is_deterministic(mode, G, n_ctas):
+    """The merge of a group's partials gives the same bits on every run: with
+    several warps per head their sums are added in a fixed order, also over
+    more units than one merge pass takes (300 units of one step each; n_ctas 0:
+    100 units and the cooperative merge)."""
+    w = small("q4_0", G, 1, [19200], outlier="student_t", q_post=1 / 16, q_outliers=False, n_out=8)
+    dw = kdev.build_pool(w, prefill_last=True)
+    q, _, _, _ = kdev.step_inputs(w, [0])
+    runs = [gc.decode_step(dw, 0, q[0], n_ctas=n_ctas, mode=mode) for _ in range(6)]
+    for out_f, out_bf, status, _, _ in runs:
+        assert status == 0
+        assert np.array_equal(out_f.view(np.int32), runs[0][0].view(np.int32))
+        assert torch.equal(out_bf.view(torch.int16), runs[0][1].view(torch.int16))
+
+
 @pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
 def test_kv_append_q_rotate_matches_separate_calls(fmt):
     """The combined launch writes the same pool bytes and the same rotated query."""
@@ -214,40 +231,47 @@ def test_kv_append_q_rotate_matches_separate_calls(fmt):
 
 
 @pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
-@pytest.mark.parametrize("case", ["ragged_g6", "ragged_g8", "cross_page_1025"])
+@pytest.mark.parametrize("case", ["ragged_g6", "ragged_g8", "cross_page_1025", "many_units_300"])
 def test_decode_step_matches_the_three_calls(case, fmt):
     """paged_decode_step = kv_append of the newest tokens + q_rotate + the
     combined decode: the same pool bytes and the same output bits, and the
-    output within the tolerance of the oracle."""
-    w, _ = _case(case, fmt)
-    a = kdev.build_pool(w, extra_slots=2, prefill_last=False)
-    b = kdev.build_pool(w, extra_slots=2, prefill_last=False)
-    q, k, v, pos = kdev.step_inputs(w, [0])
-    # stale bytes in the new token's row, which the step's copy of that tile may read
-    for dw in (a, b):
-        kvq.kv_append(dw.pool, 0, (-2.0 * k[0]).contiguous(), (0.5 * v[0].flip(-1)).contiguous(), pos, dw.page_table)
-    plan, info = kvq.decode_plan(a.pool.desc, a.seq_lens, a.page_table.shape[1], 0)
-    plan_d = torch.from_numpy(plan).cuda()
-    outs = []
-    for dw, fused_step in ((a, False), (b, True)):
-        ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
-        status = torch.zeros(1, dtype=torch.int32, device="cuda")
-        out_bf = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
-        out_f = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
-        if fused_step:
-            kvq.paged_decode_step(dw.pool, 0, q[0], k[0], v[0], dw.page_table, plan_d, info, ws, out_bf, out_f, status)
-        else:
-            kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table, status=status)
-            qp = kvq.q_rotate(q[0]) if kvq.rotated_q(fmt) else q[0]
-            kvq.paged_decode_attn_combined(dw.pool, 0, qp, dw.page_table, plan_d, info, ws, out_bf, out_f, status)
-        torch.cuda.synchronize()
-        assert int(status.item()) == 0
-        outs.append((out_f.cpu(), out_bf.cpu()))
-    assert torch.equal(a.pool.buf, b.pool.buf)
-    assert torch.equal(outs[0][0].view(torch.int32), outs[1][0].view(torch.int32))
-    assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
-    G = w.group
-    got = outs[1][0].numpy()
-    for bb in range(w.batch):
-        for g in range(w.n_kv_heads):
-            gc.assert_close(got[bb, g * G:(g + 1) * G], gc.oracle_group(b, 0, bb, g), f"step/{case}/{fmt}")
+    output within the tolerance of the oracle, for every plan size of the case
+    (one unit per SM: cooperative group merge; 300 units: more than can be
+    resident, so the last CTA of a group merges it, and units of one step)."""
+    w, nctas = _case(case, fmt)
+    for n_ctas in nctas:
+        a = kdev.build_pool(w, extra_slots=2, prefill_last=False)
+        b = kdev.build_pool(w, extra_slots=2, prefill_last=False)
+        q, k, v, pos = kdev.step_inputs(w, [0])
+        # stale bytes in the new token's row, which the step's copy of that tile may read
+        for dw in (a, b):
+            kvq.kv_append(dw.pool, 0, (-2.0 * k[0]).contiguous(), (0.5 * v[0].flip(-1)).contiguous(), pos,
+                          dw.page_table)
+        plan, info = kvq.decode_plan(a.pool.desc, a.seq_lens, a.page_table.shape[1], n_ctas)
+        plan_d = torch.from_numpy(plan).cuda()
+        outs = []
+        for dw, fused_step in ((a, False), (b, True)):
+            ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            out_bf = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+            out_f = torch.empty((w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
+            if fused_step:
+                kvq.paged_decode_step(dw.pool, 0, q[0], k[0], v[0], dw.page_table, plan_d, info, ws, out_bf, out_f,
+                                      status)
+            else:
+                kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table, status=status)
+                qp = kvq.q_rotate(q[0]) if kvq.rotated_q(fmt) else q[0]
+                kvq.paged_decode_attn_combined(dw.pool, 0, qp, dw.page_table, plan_d, info, ws, out_bf, out_f,
+                                               status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            outs.append((out_f.cpu(), out_bf.cpu()))
+        tag = f"step/{case}/{fmt}/nctas={n_ctas}"
+        assert torch.equal(a.pool.buf, b.pool.buf), tag
+        assert torch.equal(outs[0][0].view(torch.int32), outs[1][0].view(torch.int32)), tag
+        assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16)), tag
+        G = w.group
+        got = outs[1][0].numpy()
+        for bb in range(w.batch):
+            for g in range(w.n_kv_heads):
+                gc.assert_close(got[bb, g * G:(g + 1) * G], gc.oracle_group(b, 0, bb, g), f"{tag} b={bb} g={g}")

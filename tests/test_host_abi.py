@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("q_rotate", "kv_append", "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
-              "attn_combine", "kvq_pool_bytes", "kvq_pool_layout", "kvq_decode_plan"):
+              "attn_combine", "kvq_pool_bytes", "kvq_pool_layout", "kvq_decode_plan", "kv_append_q_rotate",
+              "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4"):
         assert n in names
 
 
