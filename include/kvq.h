@@ -9,6 +9,8 @@
  *   paged_decode_attn_{int8,q4_0,k8v4}
  *                                 split-K attention over the page table
  *   attn_combine                  merge the splits, un-rotate, write bf16 + f32
+ *   paged_decode_step_{int8,q4_0,k8v4}
+ *                                 all of the above for one layer in one launch
  *
  * Sources (web pages, cited by title and section):
  *  [Strata] "KV 沉进内存、显存减半：Strata 让 12 GB 显卡跑满 262K 上下文"
@@ -36,6 +38,9 @@
  *    entry out of range, an internal wait that gave up).  Affected tokens are
  *    skipped; nothing faults.  The caller clears it.
  *  - head_dim and page_tokens are both 256.
+ *  - Results are deterministic: the same inputs give the same output bits on
+ *    every run (paged_decode_attn_cudacore, a control, excepted: its last bits
+ *    may vary).
  */
 #ifndef KVQ_H
 #define KVQ_H
