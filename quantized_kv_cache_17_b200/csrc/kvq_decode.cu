@@ -30,6 +30,13 @@
 //    tokens with P'lo], P' = p * dV formed as an exact fp16 pair.  The score
 //    fragment layout of QK is exactly the P fragment layout PV needs.
 //  - a scale warp converts each stage's fp16 K scales to fp32 once.
+// Before the loop the QK warps stage the group's query through the (still
+// unused) hand-over ring, one head per warp.
+// paged_decode_step_*: the same kernel with the step enabled also rotates the
+// raw query on its way into the ring, and in the CTA whose unit ends each
+// (sequence, KV head) range the scale warp encodes the range's new token into
+// the pool (as kv_append would) and writes its codes into the last stage when
+// that lands.
 // CUDA-core kernel (the measured control): the same computation with fp32
 // FMAs only.
 #include <type_traits>
