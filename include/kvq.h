@@ -109,8 +109,13 @@ typedef struct {
     int64_t bytes_per_token_head; /* algorithmic K+V bytes of one token of one KV head */
 } kvq_layout;
 
-/* Pool size and layout for a descriptor.  KVQ_EINVAL / KVQ_EUNSUPPORTED on a
- * bad descriptor.  Host only; no CUDA call. */
+/* Pool size and layout for a descriptor ([Guide] "一": KV bytes = 2 x layers x
+ * KV heads x head_dim x bytes per element x context, here with the per-block
+ * scales counted: 288 B (q4_0), 528 B (int8) and 408 B (k8v4) per token of one
+ * KV head, so the 27B shape at 262,144 tokens in q4_0 needs the 4.8 GB the
+ * guide quotes; [Strata] "KV 从显存搬进内存之后发生了什么": KV kept in fixed
+ * pages reached through a table).  KVQ_EINVAL / KVQ_EUNSUPPORTED on a bad
+ * descriptor.  Host only; no CUDA call. */
 int kvq_pool_bytes(const kvq_pool_desc *desc, uint64_t *bytes);
 int kvq_pool_layout(const kvq_pool_desc *desc, kvq_layout *out);
 
@@ -124,7 +129,11 @@ int kvq_pool_layout(const kvq_pool_desc *desc, kvq_layout *out);
  * n_vec == 0 is a no-op. */
 int q_rotate(const float *q, float *q_rot, int64_t n_vec, void *stream);
 
-/* kv_append: encode n_rows new tokens into the pool of one layer.
+/* kv_append: encode n_rows new tokens into the pool of one layer ([Strata]
+ * "4-bit KV 缓存：先旋转，再压到 4-bit": K and V are rotated by the
+ * Walsh-Hadamard transform, then stored as 4-bit codes with a scale per block;
+ * [Guide] "二": the q4_0 block of 32 values; [Strata] "三种 KV 格式横向对比":
+ * the int8 and k8v4 variants).
  *  k, v      device fp32 [n_rows][n_kv_heads][256]
  *  row_seq   device int32 [n_rows] sequence of each row, or NULL (row i -> seq i)
  *  row_pos   device int32 [n_rows] token position of each row in its sequence
@@ -189,6 +198,9 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
  *             q_rotate, for int8 and k8v4 the plain query
  *  page_table device int32 [n_seq][max_pages]
  *  plan       device copy of the kvq_decode_plan array; info its host info
+ *             (an info whose workspace size differs from the one
+ *             kvq_decode_plan computes for its own unit and group counts is
+ *             rejected with KVQ_EINVAL)
  *  workspace  device, at least info->workspace_bytes; it ends with one int32
  *             arrival counter per (sequence, KV head) group that the
  *             *_combined entry points use: zero-fill the workspace once before
@@ -275,9 +287,10 @@ int paged_decode_step_k8v4(const kvq_pool *pool, int layer, const float *q, cons
  *  - The first call on each device, with that device current, looks up the
  *    array's device address (cudaGetSymbolAddress) and keeps it; make that first
  *    call before any stream capture.
- *  - Allocates nothing: no cudaMalloc, no cudaFree.  Each call clears the
- *    group arrival counters in the array (cudaMemsetAsync on `stream`) before
- *    the decode.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree.  Each call checks all of
+ *    its arguments first (KVQ_E* and no device work on a bad one), then clears
+ *    the group arrival counters in the array (cudaMemsetAsync on `stream`) and
+ *    runs the decode.
  *  - All calls share the one array: calls that overlap on the GPU (on
  *    different streams, or from different threads) race and give wrong output.
  *    Serialise them.

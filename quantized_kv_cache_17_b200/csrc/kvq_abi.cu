@@ -60,23 +60,42 @@ int check_pool(const kvq_pool *pool, int layer, PoolGeom *geo) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ECUDA; }
 
+}  // namespace
+
+// Host-side checks of a decode call, shared by every decode entry point (and
+// by the workspace-free one, which must run them before it touches its
+// scratch array).  Fills geo on success.
+int kvq::check_decode_args(int fmt, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                           int max_pages, const int32_t *plan, const kvq_plan_info *info, uint64_t workspace_bytes,
+                           const uint16_t *out_bf16, const float *out_f32, PoolGeom *geo) {
+    int rc = check_pool(pool, layer, geo);
+    if (rc) return rc;
+    if (pool->desc.fmt != fmt) return KVQ_EINVAL;
+    if (!q || !page_table || !plan || !info || max_pages <= 0) return KVQ_EINVAL;
+    if (!aligned16(q)) return KVQ_EALIGN;
+    const int G = pool->desc.n_q_heads / pool->desc.n_kv_heads;
+    if (info->group != G || info->n_kv_heads != pool->desc.n_kv_heads || info->n_units <= 0 || info->n_seq <= 0)
+        return KVQ_EINVAL;
+    if ((int64_t)max_pages * PAGE > INT32_MAX) return KVQ_EINVAL;
+    if (info->workspace_bytes != ws_bytes_for(info->n_units, G, info->n_seq * info->n_kv_heads)) return KVQ_EINVAL;
+    if (workspace_bytes < info->workspace_bytes) return KVQ_ESIZE;
+    if ((out_bf16 && !aligned16(out_bf16)) || (out_f32 && !aligned16(out_f32))) return KVQ_EALIGN;
+    if (!out_bf16 && out_f32) return KVQ_EINVAL;
+    return KVQ_OK;
+}
+
+namespace {
+
 int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                   int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                   uint64_t workspace_bytes, int32_t *status, void *stream, uint16_t *out_bf16 = nullptr,
                   float *out_f32 = nullptr, const float *k_new = nullptr, const float *v_new = nullptr) {
     PoolGeom geo;
-    int rc = check_pool(pool, layer, &geo);
+    if (!workspace) return KVQ_EINVAL;
+    if (!aligned16(workspace)) return KVQ_EALIGN;
+    const int rc = check_decode_args(fmt, pool, layer, q, page_table, max_pages, plan, info, workspace_bytes,
+                                     out_bf16, out_f32, &geo);
     if (rc) return rc;
-    if (pool->desc.fmt != fmt) return KVQ_EINVAL;
-    if (!q || !page_table || !plan || !info || !workspace || max_pages <= 0) return KVQ_EINVAL;
-    if (!aligned16(q) || !aligned16(workspace)) return KVQ_EALIGN;
-    const int G = pool->desc.n_q_heads / pool->desc.n_kv_heads;
-    if (info->group != G || info->n_kv_heads != pool->desc.n_kv_heads || info->n_units <= 0 || info->n_seq <= 0)
-        return KVQ_EINVAL;
-    if ((int64_t)max_pages * PAGE > INT32_MAX) return KVQ_EINVAL;
-    if (workspace_bytes < info->workspace_bytes) return KVQ_ESIZE;
-    if ((out_bf16 && !aligned16(out_bf16)) || (out_f32 && !aligned16(out_f32))) return KVQ_EALIGN;
-    if (!out_bf16 && out_f32) return KVQ_EINVAL;
     const int inverse = fmt == KVQ_INT8 ? 0 : 1;
     return cuda_rc(launch_decode(fmt, tc, static_cast<const uint8_t *>(pool->base), geo, layer, q, page_table,
                                  max_pages, plan, *info, workspace, status, inverse, out_bf16, out_f32,

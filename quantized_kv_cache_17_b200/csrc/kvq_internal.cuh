@@ -268,6 +268,13 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
     return *reinterpret_cast<__half2 *>(&u);
 }
 
+// Host-side checks of a decode call (kvq_abi.cu): pool, format, shapes, plan
+// info (its workspace size must be the one kvq_decode_plan computes) and the
+// given workspace size; KVQ_OK or a KVQ_E* code, with geo filled on success.
+int check_decode_args(int fmt, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                      int max_pages, const int32_t *plan, const kvq_plan_info *info, uint64_t workspace_bytes,
+                      const uint16_t *out_bf16, const float *out_f32, PoolGeom *geo);
+
 // Host launchers (defined in the .cu files).
 cudaError_t launch_q_rotate(const float *q, float *q_rot, int64_t n_vec, cudaStream_t s);
 cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer, const float *k,

@@ -46,15 +46,22 @@ extern "C" int paged_decode_attn_q4_0_noalloc(const kvq_pool *pool, int layer, c
                                               const int32_t *page_table, int max_pages, const int32_t *plan,
                                               const kvq_plan_info *info, uint16_t *out_bf16, float *out_f32,
                                               int32_t *status, void *stream) {
-    if (!info || !out_bf16) return KVQ_EINVAL;
-    if (info->n_units <= 0 || info->group <= 0 || info->n_seq <= 0 || info->n_kv_heads <= 0) return KVQ_EINVAL;
-    if (info->workspace_bytes > (uint64_t)KVQ_NOALLOC_WS_BYTES) return KVQ_ESIZE;
+    if (!out_bf16) return KVQ_EINVAL;
+    // Every argument check runs before the scratch array is touched: the
+    // counter clear below is sized from info, so an info that does not match
+    // its own plan sizes must be rejected first.
+    PoolGeom geo;
+    const int vrc = check_decode_args(KVQ_Q4_0, pool, layer, q, page_table, max_pages, plan, info,
+                                      KVQ_NOALLOC_WS_BYTES, out_bf16, out_f32, &geo);
+    if (vrc == KVQ_ESIZE) return KVQ_ESIZE;   // the plan needs more than the array holds
+    if (vrc != KVQ_OK) return vrc;
     void *ws = nullptr;
     const int rc = scratch_address(&ws);
     if (rc != KVQ_OK) return rc;
     // The array keeps the previous call's contents.  The fused merge needs its
     // per-group arrival counters at zero, so clear them on the caller's stream.
     const uint64_t counters_off = (uint64_t)info->n_units * ws_unit_floats(info->group) * sizeof(float);
+    if (counters_off > info->workspace_bytes) return KVQ_EINVAL;   // excluded by the checks above; kept as a guard
     const uint64_t counters_bytes = info->workspace_bytes - counters_off;
     if (cudaMemsetAsync(static_cast<unsigned char *>(ws) + counters_off, 0, counters_bytes,
                         static_cast<cudaStream_t>(stream)) != cudaSuccess)
