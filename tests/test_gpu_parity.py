@@ -275,3 +275,36 @@ def test_decode_step_matches_the_three_calls(case, fmt):
         for bb in range(w.batch):
             for g in range(w.n_kv_heads):
                 gc.assert_close(got[bb, g * G:(g + 1) * G], gc.oracle_group(b, 0, bb, g), f"{tag} b={bb} g={g}")
+
+
+def test_group_wait_times_out_and_recovers():
+    """Cooperative group merge with one unit of the group rejected by its plan
+    check: that CTA never counts in, the group's other CTAs give up after their
+    wait limit and report KVQ_STATUS_TIMEOUT (a bounded wait on the device, not
+    a hang), the launch completes without a fault, and once the counters are
+    zeroed again a good plan on the same workspace gives the oracle's result."""
+    w = small("q4_0", 6, 1, [19200], outlier="student_t", q_post=1 / 16, q_outliers=False, n_out=8)
+    dw = kdev.build_pool(w, prefill_last=True)
+    q, _, _, _ = kdev.step_inputs(w, [0])
+    qp = kvq.q_rotate(q[0])
+    plan, info = kvq.decode_plan(dw.pool.desc, dw.seq_lens, dw.page_table.shape[1], 0)
+    assert 2 <= info.n_units <= 148           # one group, cooperative merge
+    bad = plan.copy()
+    bad[8 + 4 * 1 + 2] += 32                  # unit 1 no longer starts on a step boundary
+    ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    out_bf = torch.empty((1, 6, 256), dtype=torch.bfloat16, device="cuda")
+    out_f = torch.empty((1, 6, 256), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.paged_decode_attn_combined(dw.pool, 0, qp, dw.page_table, torch.from_numpy(bad).cuda(), info, ws, out_bf,
+                                   out_f, status)
+    torch.cuda.synchronize()                  # completes: every wait is bounded
+    st = int(status.item())
+    assert st & kvq.STATUS_BAD_PLAN and st & kvq.STATUS_TIMEOUT
+    ws.zero_()                                # a timeout leaves the group counter set
+    status.zero_()
+    out_f.fill_(float("nan"))
+    kvq.paged_decode_attn_combined(dw.pool, 0, qp, dw.page_table, torch.from_numpy(plan).cuda(), info, ws, out_bf,
+                                   out_f, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    gc.assert_close(out_f.cpu().numpy()[0], gc.oracle_group(dw, 0, 0, 0), "after the timeout")
