@@ -92,11 +92,9 @@ typedef struct {
 /* Byte layout of the pool.  The pool is [layer][slot][kv_head] page blocks;
  * a page block is 32 tiles of 8 tokens; a tile holds, in this order, K codes,
  * K scales, V codes and V scales of its 8 tokens (offsets below).  Inside a
- * tile the K codes of a token are contiguous (16-byte chunks in an order that
- * depends on the token), each dimension's V codes for the tile's 8 tokens are
- * contiguous, and each token's scales are contiguous: the order the attention
- * kernel reads them in.  The exact element order is documented with the
- * kernels and reproduced by the tests' layout decoder. */
+ * tile, codes and scales are arranged in the register-fragment order of the
+ * attention kernel; the exact element order is documented with the kernels and
+ * reproduced by the tests' layout decoder. */
 typedef struct {
     int64_t tile_bytes;      /* bytes of one 8-token tile */
     int64_t k_codes_off;     /* offsets of the four sections inside a tile */
@@ -165,7 +163,7 @@ int kv_append_q_rotate(const kvq_pool *pool, int layer, const float *k, const fl
                        int32_t *status, void *stream);
 
 /* Split plan for a batch of sequences (host only).  A plan partitions every
- * (sequence, KV head) token range into work units of whole 128-token steps so
+ * (sequence, KV head) token range into work units of whole 64-token steps so
  * that the number of units does not exceed n_ctas (0 = one per SM of the
  * current device) and units are as even as possible; it also records, per
  * (sequence, KV head), the first unit.  seq_len: host int32 [n_seq], the

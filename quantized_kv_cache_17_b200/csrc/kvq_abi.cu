@@ -182,7 +182,7 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
     int64_t total = 0;
     for (int b = 0; b < n_seq; ++b) {
         if (seq_len[b] <= 0 || (int64_t)seq_len[b] > (int64_t)max_pages * PAGE) return KVQ_EINVAL;
-        steps[b] = (seq_len[b] + PLAN_TOKENS - 1) / PLAN_TOKENS;
+        steps[b] = (seq_len[b] + STEP_TOKENS - 1) / STEP_TOKENS;
         total += steps[b] * n_kv;
     }
     if (n_ctas == 0) {
@@ -208,7 +208,7 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
     info->n_kv_heads = n_kv;
     info->group = G;
     info->plan_len = len;
-    info->chunk_tokens = (int32_t)(c * PLAN_TOKENS);
+    info->chunk_tokens = (int32_t)(c * STEP_TOKENS);
     info->workspace_bytes = ws_bytes_for((int)n_units, G, n_seq * n_kv);
     if (!plan || plan_capacity < len) return KVQ_ESIZE;
     plan[0] = PLAN_MAGIC;
@@ -216,7 +216,7 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
     plan[2] = n_seq;
     plan[3] = n_kv;
     plan[4] = G;
-    plan[5] = (int32_t)(c * PLAN_TOKENS);
+    plan[5] = (int32_t)(c * STEP_TOKENS);
     plan[6] = plan[7] = 0;
     int32_t *units = plan + PLAN_HEADER;
     int32_t *start = units + 4 * n_units;
@@ -231,8 +231,8 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
                 const int64_t ns = base + (k < rem ? 1 : 0);
                 units[4 * u + 0] = b;
                 units[4 * u + 1] = g;
-                units[4 * u + 2] = (int32_t)(s0 * PLAN_TOKENS);
-                units[4 * u + 3] = (int32_t)std::min<int64_t>((s0 + ns) * PLAN_TOKENS, seq_len[b]);
+                units[4 * u + 2] = (int32_t)(s0 * STEP_TOKENS);
+                units[4 * u + 3] = (int32_t)std::min<int64_t>((s0 + ns) * STEP_TOKENS, seq_len[b]);
                 s0 += ns;
                 ++u;
             }

@@ -1,7 +1,7 @@
 // Device code of q_rotate and kv_append, shared by the launches that run them
 // on their own and by the decode-step kernel that runs them inside the decode:
 // the 256-point Walsh-Hadamard rotation and the q4_0 / int8 block quantisers,
-// written into the pool layout the decode reads (see kvq_internal.cuh).
+// written into the fragment-ordered pool layout.
 //
 // [Strata] "4-bit KV 缓存：先旋转，再压到 4-bit": K, V (and the query) are rotated
 // by a 256-point Hadamard transform before 4-bit storage; [Strata] "三种 KV 格式
@@ -119,64 +119,86 @@ __device__ __forceinline__ void quant_i8_lane(const float (&x)[8], int (&c)[8], 
     }
 }
 
-// ---- stores into the tile ------------------------------------------------------
-// K side, Q4: token r owns the 128 bytes at 128r; block b (dims 32b .. 32b+31)
-// is the 16-byte chunk at 16 (b ^ r) of them, word i of the chunk holds dims
-// 32b + 8i .. +7 with dim 32b + 8i + 2(n&3) + (n>>2) in nibble n.  Lane l holds
-// dims 8l .. 8l+7, i.e. the whole word i = l&3 of block b = l>>2.
+// ---- stores into the fragment-ordered tile ---------------------------------
+// K side, Q4: lane (block b = lane>>2, jl = lane&3) holds dims 32b + 8jl + e.
+// Dim 32b + 8(n&3) + (n>>2) + 2j lives in word W(r,b,j) nibble n, so element
+// e goes to word j = e>>1, nibble jl + 4(e&1).
 __device__ __forceinline__ void store_q4_kside(uint8_t *tile, int r, int lane, const int (&c)[8]) {
-    const int b = lane >> 2, i = lane & 3;
-    uint32_t w = 0;
+    const int b = lane >> 2, jl = lane & 3;
+    uint32_t w[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w |= (uint32_t)c[e] << (4 * (4 * (e & 1) + (e >> 1)));
-    *reinterpret_cast<uint32_t *>(tile + 128 * r + 16 * (b ^ r) + 4 * i) = w;
+    for (int j = 0; j < 4; ++j)
+        w[j] = ((uint32_t)c[2 * j] << (4 * jl)) | ((uint32_t)c[2 * j + 1] << (4 * jl + 16));
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] |= __shfl_xor_sync(0xffffffffu, w[j], m);
+    uint32_t mine = w[0];
+#pragma unroll
+    for (int j = 1; j < 4; ++j) if (jl == j) mine = w[j];
+    *reinterpret_cast<uint32_t *>(tile + (b >> 2) * 512 + (r * 4 + jl) * 16 + (b & 3) * 4) = mine;
 }
 
-// V side, Q4: word d (dim d, at 4d) holds the 8 tokens of the tile, token r
-// in nibble 4(r&1) + (r>>1).  Lane (block b = lane>>2, jl = lane&3) holds dims
-// 32b + 8jl + e.  Other tokens of the tile share the word, and a kv_append
-// call may write several tokens of one tile at once, so the nibble is replaced
-// with two atomic operations on the word (clear, then set), which leave the
-// other tokens' nibbles untouched whatever the order.
+// V side, Q4: word W(p,b,g) nibble n holds token 2p + (n>>2), dim 32b + g + 8(n&3).
+// Lane jl holds dims 32b + 8jl + e, i.e. g = e, n&3 = jl.  Token r fills the
+// 16-bit half (r&1) of words (r>>1, b, g) for g = 0..7.
 __device__ __forceinline__ void store_q4_vside(uint8_t *tile, int r, int lane, const int (&c)[8]) {
-    const int sh = 4 * (4 * (r & 1) + (r >> 1));
-    unsigned int *w = reinterpret_cast<unsigned int *>(tile) + lane * 8;
+    const int b = lane >> 2, jl = lane & 3;
+    uint32_t w[4];  // w[k] = half(g=2k) | half(g=2k+1) << 16
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        atomicAnd(w + e, ~(0xFu << sh));
-        atomicOr(w + e, (unsigned int)c[e] << sh);
+    for (int k = 0; k < 4; ++k)
+        w[k] = ((uint32_t)c[2 * k] << (4 * jl)) | ((uint32_t)c[2 * k + 1] << (4 * jl + 16));
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[k] |= __shfl_xor_sync(0xffffffffu, w[k], m);
+    uint32_t mine = w[0];
+#pragma unroll
+    for (int k = 1; k < 4; ++k) if (jl == k) mine = w[k];
+    const int p = r >> 1, half = r & 1;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int g = 2 * jl + t;
+        const uint16_t hv = (uint16_t)(mine >> (16 * t));
+        *reinterpret_cast<uint16_t *>(tile + (b >> 2) * 512 + (g * 4 + p) * 16 + (b & 3) * 4 + half * 2) = hv;
     }
 }
 
-// K side, I8: token r owns the 256 bytes at 256r; dims 16j .. 16j+15 are the
-// 16-byte chunk at 16 (j ^ r) of them, in dim order.  Lane l holds dims 8l ..
-// 8l+7: the half l&1 of chunk j = l>>1.
+// K side, I8: word W(r,s,j) byte n holds dim 16s + 2j + {0,1,8,9}[n].  Lane
+// (s = lane>>1, hl = lane&1) holds dims 16s + 8hl + e: word j = e>>1, byte
+// 2hl + (e&1).
 __device__ __forceinline__ void store_i8_kside(uint8_t *tile, int r, int lane, const int (&c)[8]) {
-    const int j = lane >> 1;
-    uint2 w = make_uint2(0u, 0u);
+    const int s = lane >> 1, hl = lane & 1;
+    uint32_t w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        w.x |= (uint32_t)(c[e] & 0xFF) << (8 * e);
-        w.y |= (uint32_t)(c[4 + e] & 0xFF) << (8 * e);
+    for (int j = 0; j < 4; ++j)
+        w[j] = (((uint32_t)(c[2 * j] & 0xFF)) | ((uint32_t)(c[2 * j + 1] & 0xFF) << 8)) << (16 * hl);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] |= __shfl_xor_sync(0xffffffffu, w[j], 1);
+    uint8_t *base = tile + (s >> 2) * 512 + (s & 3) * 4;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int j = 2 * hl + t;
+        *reinterpret_cast<uint32_t *>(base + (r * 4 + j) * 16) = hl ? w[2 + t] : w[t];
     }
-    *reinterpret_cast<uint2 *>(tile + 256 * r + 16 * (j ^ r) + 8 * (lane & 1)) = w;
 }
 
-// V side, I8: dim d owns the 8 bytes at 8d, token r in byte r.  Lane l holds
-// dims 8l + e.
+// V side, I8: word W(p,m,g) byte n holds token 2p + (n&1), dim 16m + g + 8(n>>1).
+// Lane (m = lane>>1, hl = lane&1) holds dims 16m + 8hl + e: g = e, byte 2hl + (r&1).
 __device__ __forceinline__ void store_i8_vside(uint8_t *tile, int r, int lane, const int (&c)[8]) {
-    uint8_t *base = tile + lane * 64 + r;
+    const int m = lane >> 1, hl = lane & 1;
+    uint8_t *base = tile + (m >> 2) * 512 + (m & 3) * 4 + 2 * hl + (r & 1) + (r >> 1) * 16;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) base[e * 8] = (uint8_t)(c[e] & 0xFF);
+    for (int g = 0; g < 8; ++g) base[g * 64] = (uint8_t)(c[g] & 0xFF);
 }
 
-// Scales: token r's fp16 block scales are contiguous, block b at 2b of them
-// (q4: 8 per token at 16r; int8: 4 per token at 8r).
 __device__ __forceinline__ void store_scale_q4(uint8_t *sc, int r, int lane, __half d) {
-    if ((lane & 3) == 0) *reinterpret_cast<__half *>(sc + 16 * r + 2 * (lane >> 2)) = d;
+    if ((lane & 3) == 0)
+        *reinterpret_cast<__half *>(sc + (r >> 1) * 32 + (lane >> 2) * 4 + (r & 1) * 2) = d;
 }
 __device__ __forceinline__ void store_scale_i8(uint8_t *sc, int r, int lane, __half d) {
-    if ((lane & 7) == 0) *reinterpret_cast<__half *>(sc + 8 * r + 2 * (lane >> 3)) = d;
+    if ((lane & 7) == 0)
+        *reinterpret_cast<__half *>(sc + (r >> 1) * 16 + (lane >> 3) * 4 + (r & 1) * 2) = d;
 }
 
 // A token's codes and fp16 block scales as one lane of the encoding warp holds

@@ -10,20 +10,35 @@
 // [Guide] "一": 24 query heads share 4 KV heads (groups of 6), so every K/V
 // tile read from HBM serves the whole group.
 //
-// The product kernel (decode_umma_kernel) runs the two contractions on the
-// fifth-generation tensor cores (tcgen05): K and V codes are unpacked once into
-// tensor memory as exact fp16 values, the query and the softmax weights are
-// the shared-memory operands, and the score and output accumulators live in
-// tensor memory; the per-block scales are applied to the fp32 block sums
-// (scores) and folded into the weights (values).  A CUDA-core kernel with the
-// same data path (decode_alu_kernel) is kept as the measured control.
-//
 // Data path (both kernels): a copy warp streams the unit's tokens in 64-token
 // steps (8 tiles, contiguous inside one page block) with 1-D bulk copies into
-// a ring of shared-memory stages guarded by full/empty mbarriers.  Each unit
-// writes one partial (o[G][256] unnormalised, m[8], l[8]; scores in log2
-// units), then, with the combine fused in, takes part in the merge of its
-// group.
+// a ring of shared-memory stages guarded by full/empty mbarriers.  At the end
+// the CTA merges its warps' softmax states in shared memory and writes one
+// partial (o[G][256] unnormalised, m[8], l[8]; scores in log2 units), then,
+// with the combine fused in, takes part in the merge of its group.
+//
+// Tensor-core kernel (the product), warp-specialised:
+//  - QK warps: the query of the group as mma.sync m16n8k16 A fragments in
+//    registers (rows = [8 heads, fp16 hi | same 8 heads, fp16 lo], k = 16
+//    dims), K codes as stored placed in fp16 words as B (cols = 8 tokens;
+//    exact subnormals, the code offset removed by one m16n8k8 per tile), the
+//    per-block K scale applied to the fp32 block sums; online softmax; hands
+//    p (and the rescale factor of each head) to its PV warp through a 2-slot
+//    shared-memory ring.
+//  - PV warps: the output accumulators o[dims][heads] in registers; rows = 16
+//    dims of V codes (exact in fp16), k = [8 tokens with P'hi | the same 8
+//    tokens with P'lo], P' = p * dV formed as an exact fp16 pair.  The score
+//    fragment layout of QK is exactly the P fragment layout PV needs.
+//  - a scale warp converts each stage's fp16 K scales to fp32 once.
+// Before the loop the QK warps stage the group's query through the (still
+// unused) hand-over ring, one head per warp.
+// paged_decode_step_*: the same kernel with the step enabled also rotates the
+// raw query on its way into the ring, and in the CTA whose unit ends each
+// (sequence, KV head) range the scale warp encodes the range's new token into
+// the pool (as kv_append would) and writes its codes into the last stage when
+// that lands.
+// CUDA-core kernel (the measured control): the same computation with fp32
+// FMAs only.
 #include <mutex>
 #include <type_traits>
 
@@ -37,10 +52,6 @@ constexpr float QSCALE = 0.09016844005556021f;  // log2(e) / sqrt(256)
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr int COMBINE_MAX_UNITS = 256;            // units per group merged in one pass of the combine
 constexpr int COMBINE_SMEM = 8 * D + 8 * COMBINE_MAX_UNITS + 24;   // floats of combine scratch
-constexpr int MH_MAX_UNITS = 256;                 // units per group on the cooperative merge path
-// floats of the cooperative merge's scratch for NTH threads (merge_head)
-__host__ __device__ constexpr int mh_smem_floats(int nth) { return MH_MAX_UNITS + (nth / 64) * D + D + 1; }
-constexpr int MH_SMEM_MAX = mh_smem_floats(16 * 32);
 
 __device__ __forceinline__ __half2 q4_lo_pair(uint32_t w) {     // nibbles 0 / 4 of each half -> c - 8
     return __hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(0x64086408u));
@@ -61,8 +72,40 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
     lo = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
 }
 
+// D = A * B (C = 0), A fragment from a 16-byte shared-memory word.
+__device__ __forceinline__ void mma_z(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "f"(0.f));
+}
+// D = A * B + D
+__device__ __forceinline__ void mma_acc(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+// D = A * B (C = 0), m16n8k8: A = rows g / g+8, k 2t, 2t+1; B = k 2t, 2t+1 of column g.
+__device__ __forceinline__ void mma_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
+}
 __device__ __forceinline__ uint32_t u4_at(const uint4 &v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ float4 lds128f(const float *p) {
+    const uint4 v = lds128(p);
+    return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+// (v0, v1) = 8 floats; pair i = floats 2i, 2i+1
+__device__ __forceinline__ float2 f2_at(const float4 &v0, const float4 &v1, int i) {
+    return i == 0 ? make_float2(v0.x, v0.y)
+                  : (i == 1 ? make_float2(v0.z, v0.w) : (i == 2 ? make_float2(v1.x, v1.y) : make_float2(v1.z, v1.w)));
 }
 __device__ __forceinline__ uint2 lds64(const void *p) {
     uint2 v;
@@ -75,23 +118,498 @@ __device__ __forceinline__ void sts128(void *p, uint4 v) {
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-core kernel: configuration
+// ---------------------------------------------------------------------------
+#ifndef KVQ_QK_WARPS
+#define KVQ_QK_WARPS 7       // QK warps per CTA (and as many PV warps)
+#endif
+
+template <int FMT> struct TcCfg {
+    using L = TileLayout<FMT>;
+    static constexpr int NQK = KVQ_QK_WARPS;
+    static constexpr int SCALE_WARP = 2 * NQK;
+    static constexpr int COPY_WARP = 2 * NQK + 1;
+    static constexpr int NTHREADS = (2 * NQK + 2) * 32;
+    static constexpr int TPI = FMT == KVQ_INT8 ? 2 : 4;         // tiles per work item (measured best)
+    static constexpr int ITEMS_PER_STAGE = 8 / TPI;
+    static constexpr int STAGE_BYTES = 8 * L::BYTES;
+    static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
+    static constexpr int DP = 2;                                // slots of each QK -> PV ring
+    // fp32 K scales of a stage: per tile, token pair t at float t*KSTRIDE (block
+    // or group j of tokens 2t, 2t+1 at 2j, 2j+1); the stride pads rows so the
+    // four pairs fall into different banks
+    static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
+    static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
+    static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
+    static constexpr int PA = 32 * 2 * TPI;                     // alpha[8] in a slot, after p of 32 lanes x 2 TPI
+    static constexpr int PSLOT = PA + 16;                       // floats: p, alpha[8], item
+    static constexpr int PITEM = PA + 8;                        // the item index (int) in a slot
+    static constexpr int OSTRIDE = D + 4;                       // row stride of the PV warps' o buffers
+    static constexpr int RING = NS * STAGE_BYTES;
+    static constexpr int OBUF = NQK * 8 * OSTRIDE + 2 * NQK * 8;   // floats of the CTA merge
+    static constexpr int MERGE = (COMBINE_SMEM > OBUF ? COMBINE_SMEM : OBUF) * 4;
+    static constexpr int DATA = RING > MERGE ? RING : MERGE;
+    static constexpr int SFOFF = (DATA + 127) & ~127;
+    static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
+    // the QK -> PV rings; before the loop, the group's query (KVQ_MAX_GROUP heads)
+    static constexpr int PRING_FLOATS = NQK * DP * PSLOT > KVQ_MAX_GROUP * D ? NQK * DP * PSLOT : KVQ_MAX_GROUP * D;
+    static constexpr int BAR_OFF = POFF + PRING_FLOATS * 4;
+    // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]; then,
+    // for a decode step, the newest token's codes and scales (5 words per lane)
+    static constexpr int TKV_OFF = (BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 15) & ~15;
+    static constexpr int TOTAL = TKV_OFF + 32 * 5 * 4;
+    static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+    // A QK warp waits on the ready barrier of the stage of its next item, which
+    // lies (NQK items later) at most this many stages ahead of its last one; a
+    // wait more than one lap of the ring ahead of the barrier's pending phase
+    // would be satisfied by an older phase of the same parity.
+    static_assert((NQK + ITEMS_PER_STAGE - 1) / ITEMS_PER_STAGE < NS, "QK item stride must stay within one ring lap");
+};
+
+// Scores are formed from the codes as stored (q4_0 nibbles 0..15, int8 codes
+// + 128 as 0..255) placed directly in the low bits of fp16 words: as fp16
+// subnormals they are the exact values code * 2^-24 (or 16 code * 2^-24 for a
+// nibble in bits 4-7), so unpacking costs one AND per two values and no
+// subtraction.  The constant offset (8 or 128) is removed by one extra small
+// MMA per tile: -OFF * sum_b dK[t][b] * Q[b], Q[b] = the query's sum over block
+// b.  Two power-of-two scales keep every fp16 operand in its normal range: the
+// query fragments carry 2^kq (kq puts the group's largest |q| in [2^12, 2^13)),
+// and scores are produced in units of 2^kb, kb = kq - KBS, removed inside the
+// softmax.  The fp32 K scales are therefore stored multiplied by 2^(24 - KBS).
+template <int FMT> struct QkCodes {
+    static constexpr bool Q4 = TileLayout<FMT>::KP == PART_Q4;
+    static constexpr float OFF = Q4 ? 8.f : 128.f;
+    static constexpr int KBS = Q4 ? 6 : 11;
+    static constexpr float KSF = Q4 ? 262144.f : 8192.f;     // 2^(24 - KBS)
+};
+
+// Scale warp: convert the fp16 K scales of one stage (8 tiles) to fp32 rows
+// (times 2^(24 - KBS)).
+template <int FMT>
+__device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float *sf, int lane) {
+    using L = TileLayout<FMT>;
+    constexpr int KSB = part_scale_bytes(L::KP);        // fp16 bytes per tile: 4 token pairs
+    constexpr int PAIR_B = KSB / 4;                     // 32 (q4) or 16 (i8) bytes per pair
+    constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
+    constexpr int CPT = KSB / 16;                       // 16-byte chunks per tile
+    constexpr float F = QkCodes<FMT>::KSF;
+    for (int c = lane; c < 8 * CPT; c += 32) {
+        const int tile = c / CPT, o = (c % CPT) * 16;
+        const int pair = o / PAIR_B, within = (o % PAIR_B) / 2;
+        const uint4 h = lds128(stage + tile * L::BYTES + L::KS + o);
+        float *dst = sf + tile * 4 * KSTRIDE + pair * KSTRIDE + within;
+        const float2 a = __half22float2(u32_as_h2(h.x)), b = __half22float2(u32_as_h2(h.y));
+        const float2 cc = __half22float2(u32_as_h2(h.z)), d = __half22float2(u32_as_h2(h.w));
+        sts128(dst, make_uint4(__float_as_uint(a.x * F), __float_as_uint(a.y * F), __float_as_uint(b.x * F),
+                               __float_as_uint(b.y * F)));
+        sts128(dst + 4, make_uint4(__float_as_uint(cc.x * F), __float_as_uint(cc.y * F), __float_as_uint(d.x * F),
+                                   __float_as_uint(d.y * F)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// QK warp: scores and online softmax for one work item (tiles A, B = 16 tokens)
+// ---------------------------------------------------------------------------
+// The PV warp multiplies p by the fp16 V scale in fp16 arithmetic (an exact
+// hi/lo pair, see PvWarp::pscale), so p dV must stay in fp16's normal range
+// even when every V scale of a sequence is tiny (down to subnormal).  The QK
+// warp therefore hands over p' = p 2^sigma instead of p, with sigma a power of
+// two set from e, the largest biased fp16 exponent of the V scales its items
+// have held so far: sigma = min(15, 29 - max(e, 1)) keeps p' and p' dV below
+// 2^14 (p <= 1/2), and the weights of the largest-scale tokens get the pair's
+// full precision.  sigma only enters the softmax reference point: the warp
+// keeps m' = m - sigma as its running max, so its l and o carry 2^sigma and
+// every merge (rescale on a new max, CTA merge, split-K combine) cancels it
+// like any other shift of the reference.  e only grows, so m' never falls.
+__device__ __forceinline__ int pv_sigma(int e) { return min(15, 29 - (e > 1 ? e : 1)); }
+
+// The largest |V scale| of the TPI tiles at tp, as fp16 bits (warp-uniform).
+// fp16 magnitudes order as integers.  Tokens past the sequence end count too
+// (their bytes are stale or zero): that can only lower sigma, never overflow.
+template <int FMT> __device__ __forceinline__ uint32_t item_v_scale_max(const uint8_t *tp, int lane) {
+    using L = TileLayout<FMT>;
+    constexpr int VSB = part_scale_bytes(L::VP);              // bytes per tile
+    constexpr int PER_LANE = TcCfg<FMT>::TPI * VSB / 32;      // 16 (q4) or 4 (int8) bytes
+    constexpr int LPT = VSB / PER_LANE;                       // lanes per tile
+    const uint8_t *src = tp + (lane / LPT) * L::BYTES + L::VS + (lane % LPT) * PER_LANE;
+    uint32_t m;
+    if constexpr (PER_LANE == 16) {
+        const uint4 h = lds128(src);
+        m = __vmaxu2(__vmaxu2(h.x & 0x7FFF7FFFu, h.y & 0x7FFF7FFFu), __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));
+    } else {
+        static_assert(PER_LANE == 4, "V scale bytes per lane");
+        m = *reinterpret_cast<const uint32_t *>(src) & 0x7FFF7FFFu;
+    }
+    return __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
+}
+
+template <int FMT> struct QkWarp {
+    using L = TileLayout<FMT>;
+    using C = TcCfg<FMT>;
+    using K = QkCodes<FMT>;
+    uint4 qa[16];          // A fragments of the 16 k-steps (scaled by 2^kq)
+    uint32_t qb_hi, qb_lo; // A fragment of the offset MMA: -OFF 2^-KBS Q[2t], Q[2t+1] of head g, hi / lo rows
+    float inv_sb;          // 2^-kb
+    float m_run, l_run;    // head g (the four lanes of a group agree)
+    float sg;              // sigma of the hand-over weights (warp-uniform); m_run is m - sigma
+    uint32_t vmax;         // largest |V scale| (fp16 bits) of the items seen
+
+    // Fragments of head g (rows g: fp16 hi, g+8: fp16 lo), k-step ks: dims
+    // 16ks + 2t, +1 (x, y) and 16ks + 2t + 8, +9 (z, w).  For 4-bit keys the
+    // second pair is divided by 16, matching its codes' 16 code * 2^-24.
+    __device__ __forceinline__ void init(const float *qg, int G, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        float mx = 0.f;
+        if (g < G) {
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {
+                const float *p = qg + g * D + 16 * ks + 2 * t;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p[0] * QSCALE), fabsf(p[1] * QSCALE)),
+                                     fmaxf(fabsf(p[8] * QSCALE), fabsf(p[9] * QSCALE))));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int kq = 0;
+        if (mx > 0.f) kq = min(max(12 - ((int)((__float_as_uint(mx) >> 23) & 255u) - 127), -60), 60);
+        const float s_lo = __int_as_float((127 + kq) << 23);
+        const float s_hi = K::Q4 ? __int_as_float((127 + kq - 4) << 23) : s_lo;
+        constexpr float M_HI = K::Q4 ? 16.f : 1.f;
+        float S[8];            // sum of the represented query over block b (units 2^kq)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) S[b] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (g < G) {
+                const float *p = qg + g * D + 16 * ks + 2 * t;
+                x[0] = (p[0] * QSCALE) * s_lo; x[1] = (p[1] * QSCALE) * s_lo;
+                x[2] = (p[8] * QSCALE) * s_hi; x[3] = (p[9] * QSCALE) * s_hi;
+            }
+            uint4 f;
+            split_pair(x[0], x[1], f.x, f.y);
+            split_pair(x[2], x[3], f.z, f.w);
+            qa[ks] = f;
+            const float2 h0 = __half22float2(u32_as_h2(f.x)), l0 = __half22float2(u32_as_h2(f.y));
+            const float2 h1 = __half22float2(u32_as_h2(f.z)), l1 = __half22float2(u32_as_h2(f.w));
+            const float r = ((h0.x + l0.x) + (h0.y + l0.y)) + M_HI * ((h1.x + l1.x) + (h1.y + l1.y));
+            S[K::Q4 ? ks >> 1 : ks >> 2] += r;
+        }
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            S[b] += __shfl_xor_sync(0xffffffffu, S[b], 1);
+            S[b] += __shfl_xor_sync(0xffffffffu, S[b], 2);
+        }
+        constexpr float CA = -K::OFF / (float)(1 << K::KBS);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int b = 0; b < 8; b += 2)
+            if (b == 2 * t && (K::Q4 || b < 4)) {
+                a0 = CA * S[b];
+                a1 = CA * S[b + 1];
+            }
+        split_pair(a0, a1, qb_hi, qb_lo);
+        inv_sb = __int_as_float((127 - (kq - K::KBS)) << 23);
+        m_run = -INFINITY;
+        l_run = 0.f;
+        sg = 0.f;
+        vmax = 0u;
+    }
+
+    // B fragment of the offset MMA for one tile: fp16 K scales of token g,
+    // blocks (groups) 2t, 2t+1; zero for the missing groups of int8 keys.
+    __device__ __forceinline__ static uint32_t kscale_frag(const uint8_t *tp, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        if constexpr (K::Q4) {
+            const uint2 w = lds64(tp + L::KS + (g >> 1) * 32 + 8 * t);
+            return __byte_perm(w.x, w.y, (g & 1) ? 0x7632u : 0x5410u);
+        } else {
+            const uint2 w = lds64(tp + L::KS + (g >> 1) * 16 + 8 * (t & 1));
+            return t < 2 ? __byte_perm(w.x, w.y, (g & 1) ? 0x7632u : 0x5410u) : 0u;
+        }
+    }
+
+    // S[head g][tokens 2t, 2t+1] of tiles A (s[0], s[1]) and B (s[2], s[3]), in
+    // units of 2^kb.
+    __device__ __forceinline__ void scores(const uint8_t *tA, const float *fA, int lane, float (&s)[4]) const {
+        const uint8_t *tB = tA + L::BYTES;
+        const float *fB = fA + C::SF_TILE;
+        const int t = lane & 3;
+        {
+            float ca[4], cb[4];
+            mma_k8(ca, qb_hi, qb_lo, kscale_frag(tA, lane));
+            mma_k8(cb, qb_hi, qb_lo, kscale_frag(tB, lane));
+            s[0] = ca[0] + ca[2];
+            s[1] = ca[1] + ca[3];
+            s[2] = cb[0] + cb[2];
+            s[3] = cb[1] + cb[3];
+        }
+        if constexpr (K::Q4) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 kA = lds128(tA + L::KC + hf * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + hf * 512 + lane * 16);
+                const float4 dA0 = lds128f(fA + t * C::KSTRIDE + 8 * hf), dA1 = lds128f(fA + t * C::KSTRIDE + 8 * hf + 4);
+                const float4 dB0 = lds128f(fB + t * C::KSTRIDE + 8 * hf), dB1 = lds128f(fB + t * C::KSTRIDE + 8 * hf + 4);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int b = 4 * hf + bb;
+                    const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
+                    const uint32_t wA2 = wA >> 8, wB2 = wB >> 8;
+                    float a[4], c[4];
+                    mma_z(a, qa[2 * b], wA & 0x000F000Fu, wA & 0x00F000F0u);
+                    mma_z(c, qa[2 * b], wB & 0x000F000Fu, wB & 0x00F000F0u);
+                    mma_acc(a, qa[2 * b + 1], wA2 & 0x000F000Fu, wA2 & 0x00F000F0u);
+                    mma_acc(c, qa[2 * b + 1], wB2 & 0x000F000Fu, wB2 & 0x00F000F0u);
+                    const float2 da = f2_at(dA0, dA1, bb), db = f2_at(dB0, dB1, bb);
+                    s[0] = fmaf(a[0] + a[2], da.x, s[0]);
+                    s[1] = fmaf(a[1] + a[3], da.y, s[1]);
+                    s[2] = fmaf(c[0] + c[2], db.x, s[2]);
+                    s[3] = fmaf(c[1] + c[3], db.y, s[3]);
+                }
+            }
+        } else {
+            const float4 dA0 = lds128f(fA + t * C::KSTRIDE), dA1 = lds128f(fA + t * C::KSTRIDE + 4);
+            const float4 dB0 = lds128f(fB + t * C::KSTRIDE), dB1 = lds128f(fB + t * C::KSTRIDE + 4);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 kA = lds128(tA + L::KC + q * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + q * 512 + lane * 16);
+                float a[4], c[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t wA = u4_at(kA, j) ^ 0x80808080u, wB = u4_at(kB, j) ^ 0x80808080u;
+                    const uint32_t a0 = __byte_perm(wA, 0u, 0x4140u), a1 = __byte_perm(wA, 0u, 0x4342u);
+                    const uint32_t b0 = __byte_perm(wB, 0u, 0x4140u), b1 = __byte_perm(wB, 0u, 0x4342u);
+                    if (j == 0) {
+                        mma_z(a, qa[4 * q], a0, a1);
+                        mma_z(c, qa[4 * q], b0, b1);
+                    } else {
+                        mma_acc(a, qa[4 * q + j], a0, a1);
+                        mma_acc(c, qa[4 * q + j], b0, b1);
+                    }
+                }
+                const float2 da = f2_at(dA0, dA1, q), db = f2_at(dB0, dB1, q);
+                s[0] = fmaf(a[0] + a[2], da.x, s[0]);
+                s[1] = fmaf(a[1] + a[3], da.y, s[1]);
+                s[2] = fmaf(c[0] + c[2], db.x, s[2]);
+                s[3] = fmaf(c[1] + c[3], db.y, s[3]);
+            }
+        }
+    }
+
+    // Scores of the TPI tiles of an item, softmax update, and the hand-over
+    // slot: p' of tile j, tokens 2t, 2t+1 at lane*2TPI + 2j, +1, and the
+    // rescale factor of head g at [PA + g].  The running max keeps one binade of
+    // headroom (it moves to max + 1 only when a score exceeds it), so the rescale
+    // factor is rarely different from 1 and p stays <= 1/2 (p' <= 2^(sigma - 1)).
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tp, const float *fp, const int (&v)[C::TPI], int lane,
+                                         float *slot) {
+        constexpr int NS2 = 2 * C::TPI;       // scores per lane: tokens 2t, 2t+1 of each tile
+        const int g = lane >> 2, t = lane & 3;
+        float s[NS2];
+#pragma unroll
+        for (int h = 0; h < C::TPI / 2; ++h) {
+            float a[4];
+            scores(tp + 2 * h * L::BYTES, fp + 2 * h * C::SF_TILE, lane, a);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[4 * h + i] = a[i];
+        }
+        if (MASK) {
+#pragma unroll
+            for (int j = 0; j < C::TPI; ++j) {
+                if (2 * t >= v[j]) s[2 * j] = -INFINITY;
+                if (2 * t + 1 >= v[j]) s[2 * j + 1] = -INFINITY;
+            }
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < NS2; ++i) mx = fmaxf(mx, s[i]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx *= inv_sb;                                          // log2 units
+        vmax = max(vmax, item_v_scale_max<FMT>(tp, lane));
+        const float m_true = m_run + sg;
+        const float m_new = mx > m_true ? mx + 1.f : m_true;  // mx is finite: every item has a valid token
+        sg = (float)pv_sigma((int)(vmax >> 10));
+        const float alpha = ex2(m_run - (m_new - sg));        // 1 when unchanged; 0 on the first item
+        l_run *= alpha;
+        m_run = m_new - sg;
+        float p[NS2];
+#pragma unroll
+        for (int i = 0; i < NS2; ++i) p[i] = ex2(fmaf(s[i], inv_sb, -m_run));
+        float ls = 0.f;
+#pragma unroll
+        for (int i = 0; i < NS2; i += 4) {
+            ls += (p[i] + p[i + 1]) + (p[i + 2] + p[i + 3]);
+            sts128(slot + lane * NS2 + i, make_uint4(__float_as_uint(p[i]), __float_as_uint(p[i + 1]),
+                                                     __float_as_uint(p[i + 2]), __float_as_uint(p[i + 3])));
+        }
+        l_run += ls;
+        slot[C::PA + g] = alpha;        // the four lanes of group g store the same value
+    }
+    // An item whose page could not be read: nothing to add, nothing to rescale.
+    __device__ __forceinline__ void skip(int lane, float *slot) {
+        if (lane < 8) slot[C::PA + lane] = 1.f;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// PV warp: o[dims][heads] += V^T P for one work item
+// ---------------------------------------------------------------------------
+template <int FMT> struct PvWarp {
+    using L = TileLayout<FMT>;
+    float o[16][4];        // m-tile mt: o[16 mt + g (+8)][heads 2t, 2t+1]
+
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    }
+
+    // B operand of the value product for one block: P' = p * dV as an exact
+    // fp16 pair (hi, lo): hi = rn(p_hi dV), r = p_hi dV - hi (exact, from the
+    // fused multiply-add), lo = rn(p_lo dV + r).
+    __device__ __forceinline__ static void pscale(uint32_t dv2, uint32_t ph, uint32_t pl, uint32_t &hi, uint32_t &lo) {
+        const __half2 d = u32_as_h2(dv2);
+        const __half2 h = __hmul2(u32_as_h2(ph), d);
+        const __half2 r = __hfma2(u32_as_h2(ph), d, __hneg2(h));
+        hi = h2_as_u32(h);
+        lo = h2_as_u32(__hfma2(u32_as_h2(pl), d, r));
+    }
+    // Block b of both tiles: A = [V of tile A tokens 2t, 2t+1 | of tile B], k =
+    // 16 tokens; B = P' of the same tokens, once with the hi and once with the
+    // lo halves of the exact fp16 pair.
+    __device__ __forceinline__ void pv_q4(int b, uint32_t wA, uint32_t wB, uint32_t dA, uint32_t dB,
+                                          uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
+        uint32_t hA, lA, hB, lB;
+        pscale(dA, phA, plA, hA, lA);
+        pscale(dB, phB, plB, hB, lB);
+        const uint4 m0 = make_uint4(h2_as_u32(q4_lo_pair(wA)), h2_as_u32(q4_hi_pair(wA)),
+                                    h2_as_u32(q4_lo_pair(wB)), h2_as_u32(q4_hi_pair(wB)));
+        const uint4 m1 = make_uint4(h2_as_u32(q4_lo_pair(wA >> 8)), h2_as_u32(q4_hi_pair(wA >> 8)),
+                                    h2_as_u32(q4_lo_pair(wB >> 8)), h2_as_u32(q4_hi_pair(wB >> 8)));
+        mma_acc(o[2 * b], m0, hA, hB);
+        mma_acc(o[2 * b + 1], m1, hA, hB);
+        mma_acc(o[2 * b], m0, lA, lB);
+        mma_acc(o[2 * b + 1], m1, lA, lB);
+    }
+    __device__ __forceinline__ void pv_i8(int q, const uint4 &wvA, const uint4 &wvB, uint32_t dA, uint32_t dB,
+                                          uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
+        uint32_t hA, lA, hB, lB;
+        pscale(dA, phA, plA, hA, lA);
+        pscale(dB, phB, plB, hB, lB);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t xa = u4_at(wvA, j) ^ 0x80808080u, xb = u4_at(wvB, j) ^ 0x80808080u;
+            const uint4 m = make_uint4(h2_as_u32(i8_pair(xa, 0x4140u)), h2_as_u32(i8_pair(xa, 0x4342u)),
+                                       h2_as_u32(i8_pair(xb, 0x4140u)), h2_as_u32(i8_pair(xb, 0x4342u)));
+            mma_acc(o[4 * q + j], m, hA, hB);
+            mma_acc(o[4 * q + j], m, lA, lB);
+        }
+    }
+
+    // Tiles A, B (consecutive) with p of their tokens 2t, 2t+1.
+    template <bool MASK>
+    __device__ __forceinline__ void two_tiles(const uint8_t *tA, int vA, int vB, int t, int lane, float pA0, float pA1,
+                                              float pB0, float pB1) {
+        const uint8_t *tB = tA + L::BYTES;
+        uint32_t phA, plA, phB, plB;     // p of tokens 2t, 2t+1 as fp16 hi + lo pairs
+        split_pair(pA0, pA1, phA, plA);
+        split_pair(pB0, pB1, phB, plB);
+        // zero the scales of tokens past the end (their bytes may hold anything)
+        const uint32_t mA = MASK ? ((2 * t < vA ? 0xFFFFu : 0u) | (2 * t + 1 < vA ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
+        const uint32_t mB = MASK ? ((2 * t < vB ? 0xFFFFu : 0u) | (2 * t + 1 < vB ? 0xFFFF0000u : 0u)) : 0xFFFFFFFFu;
+        if constexpr (L::VP == PART_Q4) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 wvA = lds128(tA + L::VC + hf * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + hf * 512 + lane * 16);
+                const uint4 eA = lds128(tA + L::VS + t * 32 + hf * 16);   // (dV[2t][b], dV[2t+1][b]), b = 4 hf + bb
+                const uint4 eB = lds128(tB + L::VS + t * 32 + hf * 16);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    pv_q4(4 * hf + bb, u4_at(wvA, bb), u4_at(wvB, bb), u4_at(eA, bb) & mA, u4_at(eB, bb) & mB, phA,
+                          plA, phB, plB);
+            }
+        } else {
+            const uint4 eA = lds128(tA + L::VS + t * 16);                 // (dV[2t][q], dV[2t+1][q]), q = 0..3
+            const uint4 eB = lds128(tB + L::VS + t * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 wvA = lds128(tA + L::VC + q * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + q * 512 + lane * 16);
+                pv_i8(q, wvA, wvB, u4_at(eA, q) & mA, u4_at(eB, q) & mB, phA, plA, phB, plB);
+            }
+        }
+    }
+
+    // Rescale (factors of heads 2t, 2t+1 from the slot) and accumulate the four
+    // tiles of an item.
+    template <bool MASK>
+    __device__ __forceinline__ void item(const uint8_t *tp, const int (&v)[TcCfg<FMT>::TPI], bool ok, int lane,
+                                         const float4 (&pv)[TcCfg<FMT>::TPI / 2], float2 al) {
+        const int t = lane & 3;
+        if (__any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                o[i][0] *= al.x; o[i][2] *= al.x;
+                o[i][1] *= al.y; o[i][3] *= al.y;
+            }
+        }
+        if (!ok) return;
+#pragma unroll
+        for (int h = 0; h < TcCfg<FMT>::TPI / 2; ++h)
+            two_tiles<MASK>(tp + 2 * h * L::BYTES, v[2 * h], v[2 * h + 1], t, lane, pv[h].x, pv[h].y, pv[h].z, pv[h].w);
+    }
+
+    // Write this warp's o, heads 2t, 2t+1 scaled by sc0, sc1, to b[8][OSTRIDE]
+    // (a row stride of 260 floats keeps the stores of a warp on distinct banks).
+    __device__ __forceinline__ void store_scaled(float *b, float sc0, float sc1, int lane) const {
+        const int g = lane >> 2, t = lane & 3;
+        float *r0 = b + (2 * t) * TcCfg<FMT>::OSTRIDE + g, *r1 = r0 + TcCfg<FMT>::OSTRIDE;
+#pragma unroll
+        for (int mt = 0; mt < 16; ++mt) {
+            r0[16 * mt] = o[mt][0] * sc0;
+            r1[16 * mt] = o[mt][1] * sc1;
+            r0[16 * mt + 8] = o[mt][2] * sc0;
+            r1[16 * mt + 8] = o[mt][3] * sc1;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
 // CUDA-core compute policy (control).  Lane l owns 8 dims of K and 8 dims of V
 // for all heads; partial scores are reduced across the warp by a butterfly
 // reduce-scatter so that lane l ends with tokens l/4, heads 2(l%4), 2(l%4)+1.
 // ---------------------------------------------------------------------------
 template <int FMT, int GT> struct AluCompute {
     using L = TileLayout<FMT>;
+    static constexpr int TPI = 1;
     float qr[GT][8];
     float o[GT][8];
     float m_run[2], l_run[2];   // heads 2(l%4), 2(l%4)+1
     float *p_s;                 // warp-private [8 tokens][8 heads]
 
-    // Lane l owns dims 8l .. 8l+7 of K and of V.  Dim of K element n (nibble n
-    // of the lane's q4 word, byte n of its int8 bytes) and of V element e.
-    __device__ __forceinline__ static int kdim(int lane, int n) {
-        return L::KP == PART_Q4 ? 8 * lane + 2 * (n & 3) + (n >> 2) : 8 * lane + n;
+    __device__ __forceinline__ static int kdim(int lane, int n) {   // dim of this lane's K element n
+        if (L::KP == PART_Q4) {
+            const int b = lane >> 2, j = lane & 3;
+            return 32 * b + 8 * (n & 3) + (n >> 2) + 2 * j;
+        } else {
+            const int s = 2 * (lane >> 2) + (n >> 2), j = lane & 3;
+            const int nb = n & 3;
+            return 16 * s + 2 * j + (nb & 1) + 8 * (nb >> 1);
+        }
     }
-    __device__ __forceinline__ static int vdim(int lane, int e) { return 8 * lane + e; }
+    __device__ __forceinline__ static int vdim(int lane, int e) {   // dim of this lane's V element e
+        if (L::VP == PART_Q4) {
+            const int b = lane >> 2, g = 2 * (lane & 3) + (e >> 2);
+            return 32 * b + g + 8 * (e & 3);
+        } else {
+            const int m = 2 * (lane >> 2) + (e >> 2), g = 2 * (lane & 3) + ((e >> 1) & 1);
+            return 16 * m + g + 8 * (e & 1);
+        }
+    }
 
     __device__ __forceinline__ void init(const float *qg, int G, int lane, float *pbuf) {
 #pragma unroll
@@ -124,19 +642,22 @@ template <int FMT, int GT> struct AluCompute {
             float kv[8];
             float dk;
             if constexpr (L::KP == PART_Q4) {
-                const int b = lane >> 2;
-                const uint32_t w = lds32(tp + L::KC + 128 * r + 16 * (b ^ r) + 4 * (lane & 3));
+                const int b = lane >> 2, j = lane & 3;
+                const uint32_t w = lds32(tp + L::KC + (b >> 2) * 512 + (r * 4 + j) * 16 + (b & 3) * 4);
 #pragma unroll
                 for (int n = 0; n < 8; ++n) kv[n] = q4f(w, n);
-                dk = __half2float(*reinterpret_cast<const __half *>(tp + L::KS + 16 * r + 2 * b));
+                dk = __half2float(*reinterpret_cast<const __half *>(tp + L::KS + (r >> 1) * 32 + b * 4 + (r & 1) * 2));
             } else {
-                const uint2 w = lds64(tp + L::KC + 256 * r + 16 * ((lane >> 1) ^ r) + 8 * (lane & 1));
+                const int j = lane & 3;
 #pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    kv[n] = i8f(w.x, n);
-                    kv[4 + n] = i8f(w.y, n);
+                for (int hs = 0; hs < 2; ++hs) {
+                    const int s = 2 * (lane >> 2) + hs;
+                    const uint32_t w = lds32(tp + L::KC + (s >> 2) * 512 + (r * 4 + j) * 16 + (s & 3) * 4);
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) kv[4 * hs + n] = i8f(w, n);
                 }
-                dk = __half2float(*reinterpret_cast<const __half *>(tp + L::KS + 8 * r + 2 * (lane >> 3)));
+                const int q = (lane >> 2) >> 1;
+                dk = __half2float(*reinterpret_cast<const __half *>(tp + L::KS + (r >> 1) * 16 + q * 4 + (r & 1) * 2));
             }
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
@@ -197,28 +718,33 @@ template <int FMT, int GT> struct AluCompute {
         p_s[r * 8 + h0] = p[0];
         p_s[r * 8 + h0 + 1] = p[1];
         __syncwarp();
-        // ---- values: the lane's 8 dims hold the tile's 8 tokens each ------------
-        uint32_t vw[8];
-        if constexpr (L::VP == PART_Q4) {
-            const uint4 a = lds128(tp + L::VC + 32 * lane), b = lds128(tp + L::VC + 32 * lane + 16);
-            vw[0] = a.x; vw[1] = a.y; vw[2] = a.z; vw[3] = a.w; vw[4] = b.x; vw[5] = b.y; vw[6] = b.z; vw[7] = b.w;
-        }
+        // ---- values ------------------------------------------------------------
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) {
             float vv[8];
             float dv;
             if constexpr (L::VP == PART_Q4) {
+                const int b = lane >> 2;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) vv[e] = q4f(vw[e], 4 * (rr & 1) + (rr >> 1));
-                dv = __half2float(*reinterpret_cast<const __half *>(tp + L::VS + 16 * rr + 2 * (lane >> 2)));
-            } else {
-                if ((rr & 3) == 0) {          // tokens 0-3, then 4-7: word rr / 4 of each dim's 8 bytes
+                for (int gg = 0; gg < 2; ++gg) {
+                    const int g = 2 * (lane & 3) + gg;
+                    const uint32_t w = lds32(tp + L::VC + (b >> 2) * 512 + (g * 4 + (rr >> 1)) * 16 + (b & 3) * 4);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) vw[e] = lds32(tp + L::VC + 64 * lane + 8 * e + 4 * (rr >> 2));
+                    for (int k = 0; k < 4; ++k) vv[4 * gg + k] = q4f(w, 4 * (rr & 1) + k);
                 }
+                dv = __half2float(*reinterpret_cast<const __half *>(tp + L::VS + (rr >> 1) * 32 + b * 4 + (rr & 1) * 2));
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) vv[e] = i8f(vw[e], rr & 3);
-                dv = __half2float(*reinterpret_cast<const __half *>(tp + L::VS + 8 * rr + 2 * (lane >> 3)));
+                for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+                    for (int gg = 0; gg < 2; ++gg) {
+                        const int m = 2 * (lane >> 2) + mm, g = 2 * (lane & 3) + gg;
+                        const uint32_t w = lds32(tp + L::VC + (m >> 2) * 512 + (g * 4 + (rr >> 1)) * 16 + (m & 3) * 4);
+                        vv[4 * mm + 2 * gg + 0] = i8f(w, 0 + (rr & 1));
+                        vv[4 * mm + 2 * gg + 1] = i8f(w, 2 + (rr & 1));
+                    }
+                const int q = (lane >> 2) >> 1;
+                dv = __half2float(*reinterpret_cast<const __half *>(tp + L::VS + (rr >> 1) * 16 + q * 4 + (rr & 1) * 2));
             }
             if (MASK && rr >= valid) dv = 0.f;
 #pragma unroll
@@ -421,6 +947,7 @@ __device__ __noinline__ void combine_group(const float *ws, int G, int u0, int u
 // in parallel instead of by the last one alone.  Units [u0, u0 + n); NTH
 // threads (named barrier bar_id); sm: MH_SMEM floats.
 // ---------------------------------------------------------------------------
+constexpr int MH_MAX_UNITS = 256;                 // units per group on this path
 constexpr int MH_BATCH = 8;                       // float4 loads in flight per thread
 template <int NTH>
 __device__ void merge_head(const float *ws, int G, int u0, int n, int h, int64_t out_row, int inverse_fwht,
@@ -547,7 +1074,7 @@ struct DecodeArgs {
 // the unit.
 __device__ __forceinline__ bool unit_ok(const DecodeArgs &A, int seq, int kvh, int t0, int t1, float *wsu) {
     const bool ok = A.plan[0] == PLAN_MAGIC && seq >= 0 && seq < A.plan[2] && kvh >= 0 &&
-                    kvh < A.geo.n_kv_heads && t0 >= 0 && t0 < t1 && (t0 % PLAN_TOKENS) == 0 &&
+                    kvh < A.geo.n_kv_heads && t0 >= 0 && t0 < t1 && (t0 % STEP_TOKENS) == 0 &&
                     t1 <= A.max_pages * PAGE;
     if (!ok) {
         if (threadIdx.x == 0) status_or(A.status, KVQ_STATUS_BAD_PLAN);
@@ -563,14 +1090,14 @@ __device__ __forceinline__ bool unit_ok(const DecodeArgs &A, int seq, int kvh, i
 // Copy warp: stream the unit's 64-token steps into the stage ring.  All 32
 // lanes fetch the page slots of 32 pages at a time (one load round trip per 32
 // pages instead of one per step); lane 0 waits for free stages and issues the
-// bulk copies.  before_last (optional): an mbarrier phase to wait for before
-// the last step is requested (in a decode step, the pool write of the newest
-// token, which that step holds).  Before the warp exits, every copy it issued
-// has landed.
-template <int NS, int STAGE_BYTES, int TILE_BYTES>
+// bulk copies.  Before the warp exits, every copy it issued has landed.
+struct NoHook {
+    __device__ __forceinline__ void operator()(int, int) const {}
+};
+template <int NS, int STAGE_BYTES, int TILE_BYTES, class Hook = NoHook>
 __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, uint64_t *full, uint64_t *empty,
                                           int *stage_ok, int seq, int kvh, int t0, int n_steps, int lane,
-                                          uint64_t *before_last = nullptr) {
+                                          Hook hook = Hook()) {
     const uint8_t *head_base = A.pool + (int64_t)A.layer * A.geo.layer_stride + (int64_t)kvh * A.geo.page_bytes;
     const int32_t *pt = A.page_table + (int64_t)seq * A.max_pages;
     const uint64_t pol = policy_evict_first();
@@ -586,28 +1113,29 @@ __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, ui
             my_slot = pg < A.max_pages ? __ldg(pt + pg) : -1;
         }
         const int slot = __shfl_sync(0xffffffffu, my_slot, rel & 31);
+        hook(i, lane);                 // whole warp, before step i is requested
         if (lane == 0 && !stop) {
+            ++issued;
             const int si = i % NS;
-            if (i == n_steps - 1 && before_last && !mbar_wait_bounded(before_last, 0, WAIT_LIMIT_NS))
-                status_or(A.status, KVQ_STATUS_TIMEOUT);
             if (i >= NS && !mbar_wait_bounded(&empty[si], ((i / NS) - 1) & 1, WAIT_LIMIT_NS)) {
                 status_or(A.status, KVQ_STATUS_TIMEOUT);
                 stop = true;
+                --issued;
             } else if (slot < 0 || slot >= A.geo.n_pages) {
                 status_or(A.status, KVQ_STATUS_BAD_SLOT);
                 stage_ok[si] = 0;
                 mbar_arrive(&full[si]);
-                ++issued;
             } else {
                 stage_ok[si] = 1;
                 const uint8_t *src = head_base + (int64_t)slot * A.geo.slot_stride + ((tok & 255) >> 3) * TILE_BYTES;
                 mbar_arrive_expect_tx(&full[si], STAGE_BYTES);
                 bulk_g2s(smem + si * STAGE_BYTES, src, STAGE_BYTES, &full[si], pol);
-                ++issued;
             }
         }
         __syncwarp();
     }
+    // every copy this warp issued has landed before it exits (the consumers may
+    // have stopped early on a timeout)
     if (lane == 0) {
         for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
             if (!mbar_wait_bounded(&full[i % NS], (i / NS) & 1, WAIT_LIMIT_NS)) status_or(A.status, KVQ_STATUS_TIMEOUT);
@@ -692,22 +1220,56 @@ __device__ __forceinline__ void finish_unit(const DecodeArgs &A, const float *o_
 // last stage when it lands.  The QK warps copy the query heads h = first,
 // first + stride, ... into q_s, rotating them (ROTATE) in a decode step.
 // Encode the newest token into the pool and keep its codes and scales in
-// In a decode step, one warp of the CTA whose unit ends a (sequence, KV head)
-// range encodes the range's newest token into the pool, as kv_append would,
-// and makes the write visible to the bulk copies that read the pool later (the
-// copy of the step that holds the token waits for it).  Out of line, so that
-// its registers do not shape the allocation of the warp's main loop.
+// shared memory (5 words per lane).
 template <int FMT>
-__device__ __noinline__ void step_encode_token(const DecodeArgs &A, int seq, int kvh, int pos, int lane) {
+__device__ __noinline__ void step_encode_token(const DecodeArgs &A, int seq, int kvh, int pos, uint32_t *stash,
+                                               int lane) {
     const int64_t row = ((int64_t)seq * A.geo.n_kv_heads + kvh) * D;
-    append_token<FMT>(const_cast<uint8_t *>(A.pool), A.geo, A.layer, A.k_new + row, A.v_new + row, seq, kvh, pos,
-                      A.page_table, A.max_pages, A.status, lane);
-    __threadfence();
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    float xk[8], xv[8];
+    load8(A.k_new + row + lane * 8, xk);
+    load8(A.v_new + row + lane * 8, xv);
+    const bool in_range = pos >= 0 && pos < A.max_pages * PAGE;
+    const int slot = in_range ? A.page_table[(int64_t)seq * A.max_pages + (pos >> 8)] : -1;
+    TokenCodes t;
+    quant_token<FMT>(xk, xv, lane, t);
+    uint8_t *gtile = token_tile<FMT>(const_cast<uint8_t *>(A.pool), A.geo, A.layer, slot, kvh, pos, A.status, lane);
+    if (gtile) store_token<FMT>(t, lane, pos & 7, gtile);
+    uint32_t w[5];
+    w[4] = (uint32_t)__half_as_ushort(t.dk) | ((uint32_t)__half_as_ushort(t.dv) << 16);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        w[h] = w[2 + h] = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            w[h] |= (uint32_t)(t.k[4 * h + e] & 0xFF) << (8 * e);
+            w[2 + h] |= (uint32_t)(t.v[4 * h + e] & 0xFF) << (8 * e);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 5; ++i) stash[lane * 5 + i] = w[i];
     __syncwarp();
 }
-// Warps of the softmax group copy the query heads h = first, first + stride, ... into
-// q_s, rotating them (ROTATE) in a decode step.
+// Write the stashed token into the landed stage that holds it, over the bytes
+// the copy brought (which may predate the pool store above).
+template <int FMT>
+__device__ __noinline__ void step_patch_stage(int pos, const uint32_t *stash, uint8_t *stage, int lane) {
+    TokenCodes t;
+    uint32_t w[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = stash[lane * 5 + i];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            t.k[4 * h + e] = (w[h] >> (8 * e)) & 0xFF;
+            t.v[4 * h + e] = (w[2 + h] >> (8 * e)) & 0xFF;
+        }
+    t.dk = __ushort_as_half((unsigned short)(w[4] & 0xFFFF));
+    t.dv = __ushort_as_half((unsigned short)(w[4] >> 16));
+    store_token<FMT>(t, lane, pos & 7, stage + ((pos & 63) >> 3) * TileLayout<FMT>::BYTES);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // before the stage's next bulk fill
+    __syncwarp();
+}
 template <bool ROTATE>
 __device__ __noinline__ void step_stage_query(const float *qg, float *q_s, int G, int first, int stride, int lane) {
     for (int h = first; h < G; h += stride) {
@@ -719,623 +1281,23 @@ __device__ __noinline__ void step_stage_query(const float *qg, float *q_s, int G
     }
 }
 
-
 // ---------------------------------------------------------------------------
-// Tensor-core kernel (tcgen05): configuration
+// Tensor-core kernel
 // ---------------------------------------------------------------------------
-template <int FMT> struct UmCfg {
-    using L = TileLayout<FMT>;
-    static constexpr bool KQ4 = L::KP == PART_Q4, VQ4 = L::VP == PART_Q4;
-    static constexpr int NKB = KQ4 ? 8 : 4;              // K scale blocks per token (32 or 64 dims each)
-    static constexpr int NVB = VQ4 ? 8 : 4;              // V scale blocks per token
-    static constexpr int KSPB = 16 / NKB;                // 16-dim MMA k-steps per K block
-    static constexpr int VBM = NVB / 2;                  // V blocks per 128-dim M-tile
-    static constexpr int NPV = VBM * 16;                 // value columns per M-tile: (group, block, hi/lo, 4 heads)
-    static constexpr float KOFF = KQ4 ? 8.f : 128.f;     // code offset of the K codes as stored
-    static constexpr int STEP_BYTES = 8 * L::BYTES;      // one 64-token copy step (8 tiles)
-#ifndef KVQ_UMMA_STAGES
-    static constexpr int NS = FMT == KVQ_Q4_0 ? 6 : (FMT == KVQ_INT8 ? 4 : 5);   // copy ring steps
-#else
-    static constexpr int NS = KVQ_UMMA_STAGES;
-#endif
-    // warp roles: softmax groups 0-3 (heads 0-3) and 4-7 (heads 4-7), K 8-11, V 12-15, then
-    // the copy warp and the two MMA issuers (warp 19 idles)
-    static constexpr int W_K = 8, W_V = 12, W_COPY = 16, W_QK = 17, W_PV = 18;
-    static constexpr int NTHREADS = 20 * 32;
-    static constexpr int NCT = 16 * 32;                  // threads of the unit's merge: warps 0-15
-    // tensor memory columns
-    static constexpr int T_KOP = 0;                      // K of a 128-token stage: lane = token, col = dim pair
-    static constexpr int T_SQK = 128;                    // scores: 16 columns per K block
-    static constexpr int T_VOP = T_SQK + 16 * NKB;       // 2 slots x 64: V of 64 tokens, lane = dim
-    static constexpr int T_O = T_VOP + 128;              // output accumulators: 2 M-tiles x NPV
-    static constexpr int TMEM_COLS = 512;
-    static_assert(T_O + 2 * NPV <= TMEM_COLS, "tensor memory budget");
-    // shared memory
-    static constexpr int RING = NS * STEP_BYTES;
-    static constexpr int MERGE = (COMBINE_SMEM > MH_SMEM_MAX ? COMBINE_SMEM : MH_SMEM_MAX) * 4;
-    static constexpr int DATA = RING > MERGE ? RING : MERGE;
-    static constexpr int BQK_OFF = (DATA + 1023) & ~1023;     // query operand: 16 k-steps x [16 x 16] fp16
-    static constexpr int BPV_OFF = BQK_OFF + 16 * 512;
-    static constexpr int BPV_SLOT = 2 * NPV * 256;            // (2 NPV / 8) n-groups x 128 tokens x 16 B
-    static constexpr int SIDE_OFF = BPV_OFF + 2 * BPV_SLOT;   // [2 slots][dK | dV][128 tokens] x 16 B
-    static constexpr int RED_OFF = SIDE_OFF + 2 * 2 * 128 * 16;
-    static constexpr int RED_FLOATS = 2 * 2 * 4 * 4 + 2 * 2 * 4 + 8;   // per group [2][4 warps][4] + [2][4] ints, query max
-    static constexpr int KC_OFF = RED_OFF + RED_FLOATS * 4;   // K offset terms [8 blocks][8 heads] floats
-    static constexpr int BAR_OFF = KC_OFF + 64 * 4;
-    static constexpr int NBAR = 2 * NS + 20;
-    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;       // stage_ok[NS], step_ok[2][2], tmem base, s_last
-    static constexpr int TOTAL = MISC_OFF + NS * 4 + 4 * 4 + 8;
-    static_assert(TOTAL <= 227 * 1024, "shared memory budget");
-    static_assert(2 * BPV_SLOT >= KVQ_MAX_GROUP * D * 4, "the query is staged in the value-operand buffers");
-    // instruction descriptors: scores (M = 128 tokens, N = 16) and values (M = 128 dims, N = NPV, B MN-major)
-    static constexpr uint32_t IDESC_QK = umma_idesc_f16(128, 16, 0);
-    static constexpr uint32_t IDESC_PV = umma_idesc_f16(128, NPV, 1);
-};
-
-// mbarriers of the tensor-core kernel
-struct UmBars {
-    uint64_t *full, *empty;          // [NS] copy ring
-    uint64_t *kop_full;              // [2] K dims 0-127 / 128-255 of the stage are in TMEM (K warps)
-    uint64_t *kq_done;               // [2] the score MMAs of those dims are complete (commit)
-    uint64_t *sqk_free;              // [2] both softmax groups have read those scores
-    uint64_t *side_full;             // [2] a stage's scales and step flags are in shared memory (K warps)
-    uint64_t *vop_full, *vop_free;   // [2] V of a 64-token half in TMEM / its MMAs are complete
-    uint64_t *bpv_full, *bpv_free;   // [2] P' of a stage in shared memory / its MMAs are complete
-    uint64_t *bqk_ready;             // the query operand is in shared memory
-    uint64_t *enc_done;              // decode step: the newest token is in the pool
-    uint64_t *drain;                 // [2] final commits of the two MMA issuers
-};
-
-// 4-bit codes as exact fp16 subnormals (code x 2^-24) from a word whose nibble
-// n holds element 2(n&3) + (n>>2): pairs (0,1), (2,3), (4,5), (6,7), the second
-// and fourth at 16 x code x 2^-24.
-__device__ __forceinline__ void q4_word_sub(uint32_t w, uint32_t *o) {
-    o[0] = w & 0x000F000Fu;
-    o[1] = w & 0x00F000F0u;
-    o[2] = (w >> 8) & 0x000F000Fu;
-    o[3] = (w >> 8) & 0x00F000F0u;
-}
-// int8 codes (two's complement) as exact fp16 subnormals (code + 128) x 2^-24:
-// two pairs of consecutive bytes.
-__device__ __forceinline__ void i8_word_sub(uint32_t w, uint32_t *o) {
-    const uint32_t wb = w ^ 0x80808080u;
-    o[0] = __byte_perm(wb, 0u, 0x4140u);
-    o[1] = __byte_perm(wb, 0u, 0x4342u);
-}
-// (c - 8) and c as exact fp16 values (V operand, normal numbers)
-__device__ __forceinline__ void q4_word_pairs(uint32_t w, uint32_t *o) {
-    o[0] = h2_as_u32(q4_lo_pair(w));
-    o[1] = h2_as_u32(q4_hi_pair(w));
-    o[2] = h2_as_u32(q4_lo_pair(w >> 8));
-    o[3] = h2_as_u32(q4_hi_pair(w >> 8));
-}
-__device__ __forceinline__ void i8_word_pairs(uint32_t w, uint32_t *o) {
-    const uint32_t wb = w ^ 0x80808080u;
-    o[0] = h2_as_u32(i8_pair(wb, 0x4140u));
-    o[1] = h2_as_u32(i8_pair(wb, 0x4342u));
-}
-
-// p' = 2^(x - m - PSHIFT): the running max m moves only when a score exceeds it
-// by more than RESCALE_SLACK (log2 units), so p' <= 2^(RESCALE_SLACK - PSHIFT) = 8.
-constexpr float RESCALE_SLACK = 8.f;
-constexpr float PSHIFT = 5.f;
-
-// The value weights P' = p' dV 2^sigma go to the tensor cores as fp16 (hi, lo)
-// pairs.  sigma is a power of two for the whole unit (per softmax group), set
-// from the largest V scale exponent e seen so far (sigma = 26 - max(e, 1)), so
-// that every |P'| < 8 * 2^12 stays in fp16 range and the weights of the tokens
-// with the largest scales keep the full pair precision even when all V values
-// are tiny; the output is multiplied by 2^-sigma at the end.  When a later
-// stage brings a larger scale, sigma drops and the accumulators are rescaled
-// like a moved running max.
-__device__ __forceinline__ int um_sigma(int e) { return 26 - (e > 1 ? e : 1); }
-// (2^a, 2^a) and (2^b, 2^b) as fp16 pairs with a + b = sigma, each factor in range
-__device__ __forceinline__ void um_sigma_factors(int sig, uint32_t &fa, uint32_t &fb) {
-    const int a = sig > 15 ? 15 : (sig < -14 ? -14 : sig);
-    const uint32_t ha = (uint32_t)(a + 15) << 10, hb = (uint32_t)(sig - a + 15) << 10;
-    fa = ha | (ha << 16);
-    fb = hb | (hb << 16);
-}
-
-// ---------------------------------------------------------------------------
-// Tensor-core kernel.  One CTA per plan unit, 20 warps:
-//  warps 0-7   (S) two softmax warp groups, heads 0-3 and 4-7: thread t of a
-//              group owns token t of each 128-token stage (TMEM lane t); it
-//              reads its scores from TMEM, applies the K scales and removes the
-//              code offset, runs the online softmax of its 4 heads (a running
-//              max shared by the group, moved only in steps larger than
-//              RESCALE_SLACK, the output accumulators rescaled in TMEM when it
-//              moves) and writes its part of P' = p dV (fp16 hi/lo) to shared
-//              memory.
-//  warps 8-11  (K) unpack the stage's K codes (thread = token) into TMEM as
-//              exact fp16 subnormals, dims 0-127 and 128-255 as two halves with
-//              their own barriers, and hand the token's scales to S.
-//  warps 12-15 (V) unpack the V codes of each 64-token half (thread = dims d
-//              and 128 + d) into TMEM as exact fp16 (c - offset).
-//  warp 16     copy: 64-token steps from the pool into a ring of shared-memory
-//              stages (1-D bulk copies, full / empty mbarriers).
-//  warp 17     issues the score MMAs: per K block, S[128 tokens x (group, hi/lo,
-//              4 heads)] = K (TMEM) x Q (shared memory), 8 per half stage.
-//  warp 18     issues the value MMAs: per 128-dim M-tile, O[128 dims x (group,
-//              block, hi/lo, 4 heads)] += V (TMEM) x P' (shared memory), 8 per
-//              64-token half; in a decode step it first encodes the newest token.
-// Every wait has a time limit; past it the kernel records KVQ_STATUS_TIMEOUT,
-// drains its MMAs, frees its tensor memory and finishes.
-// ---------------------------------------------------------------------------
-
-// S (both groups, 256 threads): the group's query as the score MMA's B operand,
-// [k-step][16 rows][16 dims] fp16, row n = 8 g + 4 hl + (h & 3) for head h of
-// group g = h / 4 and half hl (0 = fp16 value, 1 = residual), K-major without
-// swizzle: element (n, k) of k-step ks at ks*512 + (n/8)*256 + (k/8)*128 +
-// (n%8)*16 + (k%8)*2.  Values are q * log2(e)/16 * 2^kq / f, kq putting the
-// group's largest |value| into [2^12, 2^13) so that the fp16 residual keeps its
-// precision and f = 16 for the dims whose 4-bit codes sit at 16 x code (dim % 8
-// in {2, 3, 6, 7}), else 1.  Also the K offset terms kc[b][h] = OFF 2^-24
-// sum over block b of the represented query, which the scores subtract.
-// Returns 2^(24 - kq), the factor from the score accumulators (codes x 2^-24,
-// query x 2^kq) to log2 units.
-template <int FMT>
-__device__ __noinline__ float um_build_query(const float *q_s, int G, uint8_t *bqk, float *kc, float *red, int t) {
-    using C = UmCfg<FMT>;
-    const int warp = t >> 5, lane = t & 31;
-    float mx = 0.f;
-    for (int i = t; i < G * D; i += 256) mx = fmaxf(mx, fabsf(q_s[i] * QSCALE));
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red[warp] = mx;
-    asm volatile("bar.sync 5, 256;" ::: "memory");
-    mx = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) mx = fmaxf(mx, red[w]);
-    int kq = 0;
-    if (mx > 0.f) kq = min(max(12 - ((int)((__float_as_uint(mx) >> 23) & 255u) - 127), -60), 60);
-    const float sc = __int_as_float((127 + kq) << 23);
-    for (int wi = t; wi < 16 * 16 * 8; wi += 256) {        // 32-bit words: (k-step, row n, dim pair kp)
-        const int ks = wi >> 7, n = (wi >> 3) & 15, kp = wi & 7;
-        const int h = 4 * (n >> 3) + (n & 3), hl = (n >> 2) & 1;
-        const float f = (C::KQ4 && (kp & 1)) ? 0.0625f : 1.f;
-        float x0 = 0.f, x1 = 0.f;
-        if (h < G) {
-            x0 = ((q_s[h * D + 16 * ks + 2 * kp] * QSCALE) * sc) * f;
-            x1 = ((q_s[h * D + 16 * ks + 2 * kp + 1] * QSCALE) * sc) * f;
-        }
-        uint32_t hi, lo;
-        split_pair(x0, x1, hi, lo);
-        *reinterpret_cast<uint32_t *>(bqk + ks * 512 + (n >> 3) * 256 + (kp >> 2) * 128 + (n & 7) * 16 +
-                                      (kp & 3) * 4) = hl ? lo : hi;
-    }
-    // offset terms, summed in a fixed order from the same represented values
-    if (t < 8 * 8) {
-        const int b = t >> 3, h = t & 7;
-        float sum = 0.f;
-        if (h < G && b < C::NKB) {
-            const int bd = D / C::NKB;
-            for (int d = b * bd; d < (b + 1) * bd; d += 2) {
-                const float f = (C::KQ4 && ((d >> 1) & 1)) ? 0.0625f : 1.f;
-                uint32_t hi, lo;
-                split_pair(((q_s[h * D + d] * QSCALE) * sc) * f, ((q_s[h * D + d + 1] * QSCALE) * sc) * f, hi, lo);
-                const float2 a = __half22float2(u32_as_h2(hi)), c = __half22float2(u32_as_h2(lo));
-                sum += ((a.x + c.x) + (a.y + c.y)) / f;
-            }
-        }
-        kc[b * 8 + h] = C::KOFF * 5.9604644775390625e-08f * sum;     // OFF 2^-24 sum
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> tensor-core reads
-    asm volatile("bar.sync 5, 256;" ::: "memory");
-    return __int_as_float((127 + 24 - kq) << 23);
-}
-
-// Bounded wait by one thread; a wait past its limit records
-// KVQ_STATUS_TIMEOUT and sets `to`, and every later wait then fails at once.
-__device__ __forceinline__ bool um_wait(uint64_t *bar, uint32_t parity, const DecodeArgs &A, bool &to) {
-    if (to) return false;
-    if (!mbar_wait_bounded(bar, parity, WAIT_LIMIT_NS)) {
-        status_or(A.status, KVQ_STATUS_TIMEOUT);
-        to = true;
-        return false;
-    }
-    return true;
-}
-// The same by all 32 lanes of a warp, with one outcome for the whole warp (the
-// tensor-memory loads and stores that follow are warp-collective).
-__device__ __forceinline__ bool um_wait_warp(uint64_t *bar, uint32_t parity, const DecodeArgs &A, bool &to) {
-    bool ok = !to && mbar_wait_bounded(bar, parity, WAIT_LIMIT_NS);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-        if (!to && (threadIdx.x & 31) == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
-        to = true;
-    }
-    return ok;
-}
-
-// K: thread t unpacks token t of each stage: dims 0-127 (words [0, NW/2)) then
-// 128-255, each half into its TMEM columns once the previous stage's score MMAs
-// of that half are complete.
-template <int FMT>
-__device__ __forceinline__ void um_k_role(const DecodeArgs &A, uint8_t *smem, const UmBars &B, const int *stage_ok,
-                                          int *step_ok, uint32_t tmem, int n_steps, int n_stages, int t, bool &to) {
-    using L = TileLayout<FMT>;
-    using C = UmCfg<FMT>;
-    constexpr int NW = C::KQ4 ? 32 : 64;              // code words per token
-    constexpr int HW = NW / 2;                        // words per half (dims 0-127 / 128-255)
-    constexpr int TB = C::KQ4 ? 128 : 256;            // bytes per token
-    const int lane = t & 31, r = t & 7;
-    const uint32_t tl = tmem + ((uint32_t)(t & ~31) << 16);
-    for (int s = 0; s < n_stages; ++s) {
-        const int step = 2 * s + (t >> 6);
-        const bool has = step < n_steps;
-        const int slot = step % C::NS;
-        uint4 sk = make_uint4(0u, 0u, 0u, 0u), sv = make_uint4(0u, 0u, 0u, 0u);
-        int ok = 0;
-        const uint8_t *tile = smem + slot * C::STEP_BYTES + ((t & 63) >> 3) * L::BYTES;
-        if (has) {
-            if (!um_wait_warp(&B.full[slot], (step / C::NS) & 1, A, to)) break;
-            ok = reinterpret_cast<const volatile int *>(stage_ok)[slot];
-            if (C::KQ4) sk = lds128(tile + L::KS + 16 * r);
-            else { const uint2 x = lds64(tile + L::KS + 8 * r); sk = make_uint4(x.x, x.y, 0u, 0u); }
-            if (C::VQ4) sv = lds128(tile + L::VS + 16 * r);
-            else { const uint2 x = lds64(tile + L::VS + 8 * r); sv = make_uint4(x.x, x.y, 0u, 0u); }
-        }
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            // the chunk of 16 dims-group j sits at 16 (j ^ r): conflict-free for the warp
-            uint32_t w[HW];
-            if (has) {
-#pragma unroll
-                for (int j = 0; j < HW / 4; ++j) {
-                    const int jj = hf * (HW / 4) + j;
-                    const uint4 v = lds128(tile + L::KC + TB * r + 16 * (jj ^ r));
-                    w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
-                }
-                if (hf == 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&B.empty[slot]);
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < HW; ++j) w[j] = 0u;
-            }
-            // the previous stage's score MMAs of this half are done with its columns
-            if (s > 0 && !um_wait_warp(&B.kq_done[hf], (s - 1) & 1, A, to)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t o[32];
-                if constexpr (C::KQ4) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) q4_word_sub(w[8 * c + i], o + 4 * i);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) i8_word_sub(w[16 * c + i], o + 2 * i);
-                }
-                Tmem<32>::st(tl + C::T_KOP + 64 * hf + 32 * c, o);
-            }
-            if (hf == 1) {
-                // scales of the token, and the validity of its step, for the softmax warps
-                uint8_t *side = smem + C::SIDE_OFF + (s & 1) * 2 * 128 * 16;
-                sts128(side + 16 * t, sk);
-                sts128(side + 128 * 16 + 16 * t, sv);
-                if ((t & 63) == 0) step_ok[2 * (s & 1) + (t >> 6)] = has && ok;
-            }
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (hf == 1) mbar_arrive(&B.side_full[s & 1]);
-                mbar_arrive(&B.kop_full[hf]);
-            }
-        }
-        if (to) break;
-    }
-}
-
-// V: thread tq unpacks dims tq (M-tile 0) and 128 + tq (M-tile 1) of every
-// 64-token half into the V slot of that half.
-template <int FMT>
-__device__ __forceinline__ void um_v_role(const DecodeArgs &A, uint8_t *smem, const UmBars &B, uint32_t tmem,
-                                          int n_steps, int tq, bool &to) {
-    using L = TileLayout<FMT>;
-    using C = UmCfg<FMT>;
-    constexpr int WPD = C::VQ4 ? 1 : 2;               // code words per dim per tile
-    const int lane = tq & 31;
-    const uint32_t tl = tmem + ((uint32_t)(tq & ~31) << 16);
-    for (int i = 0; i < n_steps; ++i) {
-        const int slot = i % C::NS;
-        if (!um_wait_warp(&B.full[slot], (i / C::NS) & 1, A, to)) break;
-        const uint8_t *stage = smem + slot * C::STEP_BYTES;
-        uint32_t w0[8 * WPD], w1[8 * WPD];
-#pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-            const uint8_t *v = stage + tt * L::BYTES + L::VC;
-            if constexpr (C::VQ4) {
-                w0[tt] = lds32(v + 4 * tq);
-                w1[tt] = lds32(v + 4 * (128 + tq));
-            } else {
-                const uint2 a = lds64(v + 8 * tq), b = lds64(v + 8 * (128 + tq));
-                w0[2 * tt] = a.x; w0[2 * tt + 1] = a.y;
-                w1[2 * tt] = b.x; w1[2 * tt + 1] = b.y;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.empty[slot]);
-        if (i >= 2 && !um_wait_warp(&B.vop_free[i & 1], ((i - 2) >> 1) & 1, A, to)) break;
-        tc_fence_after();
-        uint32_t o[32];
-#pragma unroll
-        for (int j = 0; j < 8 * WPD; ++j) {
-            if constexpr (C::VQ4) q4_word_pairs(w0[j], o + 4 * j);
-            else i8_word_pairs(w0[j], o + 2 * j);
-        }
-        Tmem<32>::st(tl + C::T_VOP + 64 * (i & 1), o);
-#pragma unroll
-        for (int j = 0; j < 8 * WPD; ++j) {
-            if constexpr (C::VQ4) q4_word_pairs(w1[j], o + 4 * j);
-            else i8_word_pairs(w1[j], o + 2 * j);
-        }
-        Tmem<32>::st(tl + C::T_VOP + 64 * (i & 1) + 32, o);
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.vop_full[i & 1]);
-    }
-}
-
-// Score MMA issuer (one thread): per stage, the 8 k-steps of dims 0-127 as soon
-// as K warps have written them, then the 8 of dims 128-255.
-template <int FMT>
-__device__ __forceinline__ void um_qk_issue(const DecodeArgs &A, uint8_t *smem, const UmBars &B, uint32_t tmem,
-                                            int n_stages, bool &to) {
-    using C = UmCfg<FMT>;
-    if (!um_wait(B.bqk_ready, 0, A, to)) return;
-    const uint32_t bqk = smem_u32(smem + C::BQK_OFF);
-    for (int s = 0; s < n_stages; ++s) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            if (!um_wait(&B.kop_full[hf], s & 1, A, to)) return;
-            if (s > 0 && !um_wait(&B.sqk_free[hf], (s - 1) & 1, A, to)) return;
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int ks = 8 * hf + k;
-                umma_f16_ts(tmem + C::T_SQK + 16 * (ks / C::KSPB), tmem + C::T_KOP + 8 * ks,
-                            umma_sdesc(bqk + ks * 512, 128, 256), C::IDESC_QK, (ks % C::KSPB) != 0);
-            }
-            tc_commit(&B.kq_done[hf]);
-        }
-    }
-}
-
-// Value MMA issuer (one thread).  P' of stage s: slot s & 1, n-group g (8
-// consecutive accumulator columns) at g*2048, token k of the stage at k*16.
-template <int FMT>
-__device__ __forceinline__ void um_pv_issue(const DecodeArgs &A, uint8_t *smem, const UmBars &B, uint32_t tmem,
-                                            int n_steps, bool &to) {
-    using C = UmCfg<FMT>;
-    const uint32_t bpv = smem_u32(smem + C::BPV_OFF);
-    bool first = true;
-    for (int i = 0; i < n_steps; ++i) {
-        const int s = i >> 1;
-        if ((i & 1) == 0 && !um_wait(&B.bpv_full[s & 1], (s >> 1) & 1, A, to)) return;
-        if (!um_wait(&B.vop_full[i & 1], (i >> 1) & 1, A, to)) return;
-        tc_fence_after();
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t b = bpv + (s & 1) * C::BPV_SLOT + mt * (C::NPV / 8) * 2048 + ((i & 1) * 8 + 2 * kk) * 128;
-                umma_f16_ts(tmem + C::T_O + C::NPV * mt, tmem + C::T_VOP + 64 * (i & 1) + 32 * mt + 8 * kk,
-                            umma_sdesc(b, 128, 2048), C::IDESC_PV, !(first && kk == 0));
-            }
-        first = false;
-        tc_commit(&B.vop_free[i & 1]);
-        if ((i & 1) == 1 || i == n_steps - 1) tc_commit(&B.bpv_free[s & 1]);
-    }
-}
-
-// Group-wide OR over the 128 threads of softmax group g (named barrier 2 + g).
-__device__ __forceinline__ bool um_group_any(int g, bool v) {
-    uint32_t r;
-    if (g == 0)
-        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 2, 128, p;\n\t"
-                     "selp.u32 %0, 1, 0, q;\n\t}" : "=r"(r) : "r"((uint32_t)v) : "memory");
-    else
-        asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 3, 128, p;\n\t"
-                     "selp.u32 %0, 1, 0, q;\n\t}" : "=r"(r) : "r"((uint32_t)v) : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void um_group_sync(int g) {
-    if (g == 0) asm volatile("bar.sync 2, 128;" ::: "memory");
-    else asm volatile("bar.sync 3, 128;" ::: "memory");
-}
-
-// S: one softmax group (g = 0: heads 0-3, 1: heads 4-7).  Returns, for the
-// unit's partial, the reference m + PSHIFT of its heads (log2 units; p' =
-// 2^(x - reference)), this thread's sum of p' per head, and 2^-sigma.
-template <int FMT>
-__device__ __forceinline__ void um_s_role(const DecodeArgs &A, uint8_t *smem, const UmBars &B, const int *step_ok,
-                                          uint32_t tmem, float qsc, int t0, int t1, int n_stages, int g, int t,
-                                          float (&m)[4], float (&l)[4], float &unsig, bool &to) {
-    using C = UmCfg<FMT>;
-    const int warp = t >> 5, lane = t & 31;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    float *red = reinterpret_cast<float *>(smem + C::RED_OFF) + g * (2 * 4 * 4 + 2 * 4);
-    int *red_e = reinterpret_cast<int *>(red + 2 * 4 * 4);          // [2][4] exponent maxima
-    const float *kc = reinterpret_cast<const float *>(smem + C::KC_OFF);
-    float mref[4];        // m + PSHIFT, or 0 while m is still -inf (no valid token yet)
-#pragma unroll
-    for (int h = 0; h < 4; ++h) { m[h] = -INFINITY; l[h] = 0.f; mref[h] = 0.f; }
-    int e_cur = 0;
-    uint32_t fa, fb;
-    um_sigma_factors(um_sigma(0), fa, fb);
-    for (int s = 0; s < n_stages; ++s) {
-        bool ok = um_wait_warp(&B.side_full[s & 1], (s >> 1) & 1, A, to);
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        uint4 skk = make_uint4(0u, 0u, 0u, 0u), svv = make_uint4(0u, 0u, 0u, 0u);
-        bool valid = false;
-        if (ok) {
-            const uint8_t *side = smem + C::SIDE_OFF + (s & 1) * 2 * 128 * 16;
-            skk = lds128(side + 16 * t);
-            svv = lds128(side + 128 * 16 + 16 * t);
-            valid = step_ok[2 * (s & 1) + (t >> 6)] != 0 && t0 + 128 * s + t < t1;
-        }
-        // scores of the group's heads: x_h = sum_b dK_b 2^-kq (S_b[hi h] + S_b[lo h] - kc[b][h])
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            ok = ok && um_wait_warp(&B.kq_done[hf], s & 1, A, to);
-            if (ok) {
-                tc_fence_after();
-                constexpr int NB = C::NKB / 2;                 // K blocks per half
-                uint32_t r[NB][8];
-#pragma unroll
-                for (int bb = 0; bb < NB; ++bb) {
-                    uint32_t (&rb)[8] = r[bb];
-                    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                                 : "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]),
-                                   "=r"(rb[6]), "=r"(rb[7])
-                                 : "r"(tl + C::T_SQK + 16 * (NB * hf + bb) + 8 * g)
-                                 : "memory");
-                }
-                tc_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&B.sqk_free[hf]);
-#pragma unroll
-                for (int bb = 0; bb < NB; ++bb) {
-                    const int b = NB * hf + bb;
-                    const float dk = __half2float(__ushort_as_half((unsigned short)(u4_at(skk, b >> 1) >> (16 * (b & 1))))) * qsc;
-                    const float4 c = *reinterpret_cast<const float4 *>(kc + 8 * b + 4 * g);
-                    x[0] = fmaf((__uint_as_float(r[bb][0]) + __uint_as_float(r[bb][4])) - c.x, dk, x[0]);
-                    x[1] = fmaf((__uint_as_float(r[bb][1]) + __uint_as_float(r[bb][5])) - c.y, dk, x[1]);
-                    x[2] = fmaf((__uint_as_float(r[bb][2]) + __uint_as_float(r[bb][6])) - c.z, dk, x[2]);
-                    x[3] = fmaf((__uint_as_float(r[bb][3]) + __uint_as_float(r[bb][7])) - c.w, dk, x[3]);
-                }
-            } else {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&B.sqk_free[hf]);
-            }
-        }
-        if (!valid) {
-            svv = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) x[h] = -INFINITY;
-        }
-        // largest V scale exponent of the token (fp16 magnitudes order as integers)
-        uint32_t vm = __vmaxu2(__vmaxu2(svv.x & 0x7FFF7FFFu, svv.y & 0x7FFF7FFFu),
-                               __vmaxu2(svv.z & 0x7FFF7FFFu, svv.w & 0x7FFF7FFFu));
-        vm = max(vm & 0xFFFFu, vm >> 16);
-        const int e_tok = (int)(vm >> 10);
-        // the running max moves only past the slack, sigma only for a larger
-        // scale exponent; both checks, and a timed-out wait, are decided for the
-        // whole group
-        bool need = e_tok > e_cur;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) need |= x[h] > m[h] + RESCALE_SLACK;
-        if (um_group_any(g, need || to)) {
-            if (um_group_any(g, to)) { to = true; break; }
-            float mx[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                mx[h] = x[h];
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
-            }
-            const int ew = (int)__reduce_max_sync(0xffffffffu, (unsigned)e_tok);
-            float *rr = red + (s & 1) * 16;
-            if (lane < 4) rr[warp * 4 + lane] = lane == 0 ? mx[0] : (lane == 1 ? mx[1] : (lane == 2 ? mx[2] : mx[3]));
-            if (lane == 0) red_e[(s & 1) * 4 + warp] = ew;
-            um_group_sync(g);
-            const int *re = red_e + (s & 1) * 4;
-            const int e_new = max(e_cur, max(max(re[0], re[1]), max(re[2], re[3])));
-            const int sig_old = um_sigma(e_cur), sig_new = um_sigma(e_new);
-            const float sc = __int_as_float((127 + sig_new - sig_old) << 23);   // 2^(sigma_new - sigma_old) <= 1
-            e_cur = e_new;
-            um_sigma_factors(sig_new, fa, fb);
-            float alpha[4];
-            bool moved = sig_new != sig_old;
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float M = fmaxf(fmaxf(rr[h], rr[4 + h]), fmaxf(rr[8 + h], rr[12 + h]));
-                const float mn = M > m[h] ? M : m[h];
-                alpha[h] = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
-                moved |= mn != m[h] && m[h] != -INFINITY;
-                m[h] = mn;
-                mref[h] = mn == -INFINITY ? 0.f : mn + PSHIFT;
-                l[h] *= alpha[h];
-                alpha[h] *= sc;              // the accumulators also carry 2^sigma
-            }
-            // rescale the group's output columns once every earlier value MMA is
-            // complete (the first stage has nothing accumulated yet)
-            if (s > 0 && moved) {
-                um_wait_warp(&B.bpv_free[(s - 1) & 1], ((s - 1) >> 1) & 1, A, to);   // a timeout ends the loop at the next stage
-                tc_fence_after();
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    const uint32_t ta = tl + C::T_O + C::NPV * mt + g * (C::NPV / 2);
-                    if constexpr (C::NPV / 2 == 32) {
-                        uint32_t r[32];
-                        Tmem<32>::ld(ta, r);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha[j & 3]);
-                        Tmem<32>::st(ta, r);
-                    } else {
-                        uint32_t r[16];
-                        Tmem<16>::ld(ta, r);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha[j & 3]);
-                        Tmem<16>::st(ta, r);
-                    }
-                }
-                tc_wait_st();
-            }
-            um_group_sync(g);            // the reduction slots are read before the next stage writes them
-        }
-        // p' = 2^(x - m - PSHIFT); masked tokens give 0
-        float p[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            p[h] = ex2(x[h] - mref[h]);
-            l[h] += p[h];
-        }
-        // the token's V scales times 2^sigma (exact: two power-of-two products)
-        svv.x = h2_as_u32(__hmul2(__hmul2(u32_as_h2(svv.x), u32_as_h2(fa)), u32_as_h2(fb)));
-        svv.y = h2_as_u32(__hmul2(__hmul2(u32_as_h2(svv.y), u32_as_h2(fa)), u32_as_h2(fb)));
-        if (C::NVB > 4) {
-            svv.z = h2_as_u32(__hmul2(__hmul2(u32_as_h2(svv.z), u32_as_h2(fa)), u32_as_h2(fb)));
-            svv.w = h2_as_u32(__hmul2(__hmul2(u32_as_h2(svv.w), u32_as_h2(fa)), u32_as_h2(fb)));
-        }
-        // P' = p' dV 2^sigma as exact fp16 (hi, lo) pairs into slot s & 1
-        if (s >= 2) um_wait_warp(&B.bpv_free[s & 1], ((s - 2) >> 1) & 1, A, to);   // a timeout ends the loop next stage
-        uint32_t ph0, pl0, ph1, pl1;
-        split_pair(p[0], p[1], ph0, pl0);
-        split_pair(p[2], p[3], ph1, pl1);
-        uint8_t *bp = smem + C::BPV_OFF + (s & 1) * C::BPV_SLOT + 16 * t;
-#pragma unroll
-        for (int b = 0; b < C::NVB; ++b) {
-            const uint32_t dvw = u4_at(svv, b >> 1);
-            const __half2 dv = u32_as_h2(__byte_perm(dvw, dvw, (b & 1) ? 0x3232u : 0x1010u));    // (dV_b, dV_b)
-            const __half2 h0 = __hmul2(u32_as_h2(ph0), dv), h1 = __hmul2(u32_as_h2(ph1), dv);
-            const __half2 l0 = __hfma2(u32_as_h2(pl0), dv, __hfma2(u32_as_h2(ph0), dv, __hneg2(h0)));
-            const __half2 l1 = __hfma2(u32_as_h2(pl1), dv, __hfma2(u32_as_h2(ph1), dv, __hneg2(h1)));
-            const int mt = b / C::VBM, bl = b % C::VBM;
-            const int ng = mt * (C::NPV / 8) + g * C::VBM + bl;          // n-group (group, block): hi h0-3, lo h0-3
-            sts128(bp + ng * 2048, make_uint4(h2_as_u32(h0), h2_as_u32(h1), h2_as_u32(l0), h2_as_u32(l1)));
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // generic writes -> tensor-core reads
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.bpv_full[s & 1]);
-    }
-    unsig = __int_as_float((127 - um_sigma(e_cur)) << 23);
-}
-
 template <int FMT, bool FUSED, bool STEP = false>
-__global__ void __launch_bounds__(UmCfg<FMT>::NTHREADS, 1) decode_umma_kernel(const __grid_constant__ DecodeArgs A) {
+__global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(const __grid_constant__ DecodeArgs A) {
     static_assert(!STEP || FUSED, "the decode step merges in the kernel");
     using L = TileLayout<FMT>;
-    using C = UmCfg<FMT>;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    using C = TcCfg<FMT>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *ready = full + C::NS;            // fp32 K scales of the stage are written
+    uint64_t *empty = ready + C::NS;           // every item of the stage is done
+    uint64_t *p_full = empty + C::NS;          // QK -> PV slot written
+    uint64_t *p_empty = p_full + C::NQK * C::DP;
+    int *stage_ok = reinterpret_cast<int *>(p_empty + C::NQK * C::DP);
+    __shared__ int s_last;
+
     grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u = blockIdx.x;
@@ -1344,153 +1306,186 @@ __global__ void __launch_bounds__(UmCfg<FMT>::NTHREADS, 1) decode_umma_kernel(co
     const int G = A.G;
     const int n_units = A.plan[1];
     float *wsu = A.ws + (size_t)u * ws_unit_floats(G);
-    if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;           // the whole CTA, before anything is allocated
+    if (!unit_ok(A, seq, kvh, t0, t1, wsu)) return;
     const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
-    const int n_stages = (n_steps + 1) / 2;
-
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-    UmBars B;
-    B.full = bars;
-    B.empty = bars + C::NS;
-    uint64_t *nb = bars + 2 * C::NS;
-    B.kop_full = nb;
-    B.kq_done = nb + 2;
-    B.sqk_free = nb + 4;
-    B.side_full = nb + 6;
-    B.vop_full = nb + 8;
-    B.vop_free = nb + 10;
-    B.bpv_full = nb + 12;
-    B.bpv_free = nb + 14;
-    B.drain = nb + 16;
-    B.bqk_ready = nb + 18;
-    B.enc_done = nb + 19;
-    int *stage_ok = reinterpret_cast<int *>(smem + C::MISC_OFF);
-    int *step_ok = stage_ok + C::NS;                           // [2 stage slots][2 halves]
-    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(step_ok + 4);
-    int *s_last = reinterpret_cast<int *>(tmem_base + 1);
+    const int n_items = (t1 - t0 + C::TPI * TILE - 1) / (C::TPI * TILE);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NS; ++i) {
-            mbar_init(&B.full[i], 1);
-            mbar_init(&B.empty[i], 6);                       // 2 K warps + 4 V warps read each step
+            mbar_init(&full[i], 1);
+            mbar_init(&ready[i], 32);                    // every lane of the scale warp arrives
+            mbar_init(&empty[i], 32 * C::ITEMS_PER_STAGE);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&B.kop_full[i], 4);
-            mbar_init(&B.kq_done[i], 1);
-            mbar_init(&B.sqk_free[i], 8);
-            mbar_init(&B.side_full[i], 4);
-            mbar_init(&B.vop_full[i], 4);
-            mbar_init(&B.vop_free[i], 1);
-            mbar_init(&B.bpv_full[i], 8);
-            mbar_init(&B.bpv_free[i], 1);
-            mbar_init(&B.drain[i], 1);
+        for (int i = 0; i < C::NQK * C::DP; ++i) {      // every lane of the QK / PV warp arrives
+            mbar_init(&p_full[i], 32);
+            mbar_init(&p_empty[i], 32);
         }
-        mbar_init(B.bqk_ready, 8);
-        mbar_init(B.enc_done, 1);
         fence_mbar_init();
     }
-    if (warp == C::W_QK) tmem_alloc(tmem_base, C::TMEM_COLS);
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_base;
-    // decode step: the CTA whose unit ends the (sequence, KV head) range appends its newest token
+    // decode step: the last CTA of the group appends the group's newest token
     const bool appends = STEP && u == A.plan[PLAN_HEADER + 4 * n_units + seq * A.geo.n_kv_heads + kvh + 1] - 1;
-    bool to = false;
 
-    if (warp == C::W_COPY) {
-        copy_loop<C::NS, C::STEP_BYTES, L::BYTES>(A, smem, B.full, B.empty, stage_ok, seq, kvh, t0, n_steps, lane,
-                                                  appends ? B.enc_done : nullptr);
+    if (warp == C::COPY_WARP) {
+        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
         return;
     }
-    if (warp > C::W_PV) return;                                  // spare warp
-    if (warp == C::W_QK || warp == C::W_PV) {
-        if (warp == C::W_PV && appends) {
-            step_encode_token<FMT>(A, seq, kvh, t1 - 1, lane);
-            if (lane == 0) mbar_arrive(B.enc_done);
-        }
-        if (lane == 0) {
-            if (warp == C::W_QK) um_qk_issue<FMT>(A, smem, B, tmem, n_stages, to);
-            else um_pv_issue<FMT>(A, smem, B, tmem, n_steps, to);
-            // every MMA this thread issued is complete before the memory is freed
-            tc_commit(&B.drain[warp - C::W_QK]);
-            bool dto = false;
-            um_wait(&B.drain[warp - C::W_QK], 0, A, dto);
-        }
-        __syncwarp();
-        asm volatile("bar.sync 4, 320;" ::: "memory");       // with the softmax warps: tensor memory is idle
-        if (warp == C::W_QK) {
-            tc_fence_after();
-            tmem_dealloc(tmem, C::TMEM_COLS);
-        }
-        return;
-    }
-
-    if (warp < C::W_K) {
-        const int g = warp >> 2, t = threadIdx.x & 127;
-        const float *qg = A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D;
-        float *q_s = reinterpret_cast<float *>(smem + C::BPV_OFF);       // free until the first P'
-        step_stage_query<STEP && Fmt<FMT>::KROT>(qg, q_s, G, warp, 8, lane);
-        asm volatile("bar.sync 5, 256;" ::: "memory");
-        const float qsc = um_build_query<FMT>(q_s, G, smem + C::BQK_OFF, reinterpret_cast<float *>(smem + C::KC_OFF),
-                                              reinterpret_cast<float *>(smem + C::RED_OFF) + 2 * (2 * 4 * 4 + 2 * 4),
-                                              threadIdx.x);
-        if (lane == 0) mbar_arrive(B.bqk_ready);
-        float m[4], l[4], unsig;
-        um_s_role<FMT>(A, smem, B, step_ok, tmem, qsc, t0, t1, n_stages, g, t, m, l, unsig, to);
-        // the unit's partial: o from the accumulators once the last value MMA is done
-        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        um_wait_warp(&B.bpv_free[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1, A, to);
-        tc_fence_after();
-        float o0[4], o1[4];
-        {
-            const int bl = ((warp & 3) * 32) / (256 / C::NVB);      // V block of dim t inside its M-tile
-            uint32_t r[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                           "=r"(r[7])
-                         : "r"(tl + C::T_O + g * (C::NPV / 2) + 8 * bl)
-                         : "memory");
-            tc_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 4; ++h) o0[h] = (__uint_as_float(r[h]) + __uint_as_float(r[4 + h])) * unsig;
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                           "=r"(r[7])
-                         : "r"(tl + C::T_O + C::NPV + g * (C::NPV / 2) + 8 * bl)
-                         : "memory");
-            tc_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 4; ++h) o1[h] = (__uint_as_float(r[h]) + __uint_as_float(r[4 + h])) * unsig;
-        }
-        tc_fence_before();
-        asm volatile("bar.arrive 4, 320;" ::: "memory");       // tensor memory may be freed
-        // l: sum over the 128 tokens of the group
-        float *red = reinterpret_cast<float *>(smem + C::RED_OFF) + g * (2 * 4 * 4 + 2 * 4);
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
-        um_group_sync(g);
-        if (lane < 4) red[(warp & 3) * 4 + lane] = lane == 0 ? l[0] : (lane == 1 ? l[1] : (lane == 2 ? l[2] : l[3]));
-        um_group_sync(g);
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-            if (4 * g + h < G) {
-                wsu[(4 * g + h) * D + t] = o0[h];
-                wsu[(4 * g + h) * D + 128 + t] = o1[h];
+    if (warp == C::SCALE_WARP) {
+        uint32_t *stash = reinterpret_cast<uint32_t *>(smem + C::TKV_OFF);
+        if (appends) step_encode_token<FMT>(A, seq, kvh, t1 - 1, stash, lane);
+        for (int i = 0; i < n_steps; ++i) {
+            const int si = i % C::NS;
+            if (!mbar_wait_bounded(&full[si], (i / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
             }
-        if (t < 4) {
-            const float mv = t == 0 ? m[0] : (t == 1 ? m[1] : (t == 2 ? m[2] : m[3]));
-            wsu[G * D + 4 * g + t] = mv + PSHIFT;
-            wsu[G * D + 8 + 4 * g + t] = (red[t] + red[4 + t]) + (red[8 + t] + red[12 + t]);
+            if (appends && i == n_steps - 1 && stage_ok[si])    // the stage that holds the newest token
+                step_patch_stage<FMT>(t1 - 1, stash, smem + si * C::STAGE_BYTES, lane);
+            if (stage_ok[si])
+                convert_stage_scales<FMT>(smem + si * C::STAGE_BYTES,
+                                          reinterpret_cast<float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES), lane);
+            __syncwarp();
+            mbar_arrive(&ready[si]);
         }
-    } else if (warp < C::W_V) {
-        um_k_role<FMT>(A, smem, B, stage_ok, step_ok, tmem, n_steps, n_stages, threadIdx.x - 32 * C::W_K, to);
-    } else {
-        um_v_role<FMT>(A, smem, B, tmem, n_steps, threadIdx.x - 32 * C::W_V, to);
+        return;
     }
-    publish_unit<FUSED, C::NCT>(A, seq, kvh, n_units, s_last, smem);
+
+    float *pring = reinterpret_cast<float *>(smem + C::POFF);
+    constexpr int NCT = 2 * C::NQK * 32;       // merge threads: QK + PV warps
+    const bool is_qk = warp < C::NQK;
+    const int pw = is_qk ? warp : warp - C::NQK;    // pair index
+    QkWarp<FMT> qk;
+    PvWarp<FMT> pv;
+    // Pair pw takes items pw, pw + NQK, ... (item `it` = tiles 4 it .. 4 it + 3 =
+    // half of stage it / 2); the QK warp passes the item index, or -1 at the end,
+    // to its PV warp with the scores.  (Handing items out from a shared counter
+    // instead measured slower on long units.)
+    if (is_qk) {
+        const float *qg = A.q + ((int64_t)seq * A.n_q_heads + (int64_t)kvh * G) * D;
+        // The group's query goes through the (still unused) hand-over ring, one
+        // head per QK warp: a warp that loads all G heads itself waits longer
+        // while the first stages flood the memory system.  A decode step
+        // rotates the raw query on the way, as q_rotate would.
+        step_stage_query<STEP && Fmt<FMT>::KROT>(qg, pring, G, pw, C::NQK, lane);
+        asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+        qk.init(pring, G, lane);
+        asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
+        for (int k = 0;; ++k) {
+            const int slot = k % C::DP;
+            float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
+            if (k >= C::DP && !mbar_wait_bounded(&p_empty[pw * C::DP + slot], ((k / C::DP) - 1) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            const int it = pw + C::NQK * k;
+            if (it >= n_items) {                       // no work left: tell the PV warp
+                if (lane == 0) reinterpret_cast<int *>(ps)[C::PITEM] = -1;
+                mbar_arrive(&p_full[pw * C::DP + slot]);
+                break;
+            }
+            const int st = it / C::ITEMS_PER_STAGE, si = st % C::NS, within = it % C::ITEMS_PER_STAGE;
+            // ready implies the stage's bulk copy has landed (the scale warp waited for it)
+            if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            const int tok = t0 + it * C::TPI * TILE;
+            int v[C::TPI];
+#pragma unroll
+            for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
+            if (stage_ok[si]) {
+                const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
+                const float *fp = reinterpret_cast<const float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES) +
+                                  within * C::TPI * C::SF_TILE;
+                if (v[C::TPI - 1] == TILE) qk.template item<false>(tp, fp, v, lane, ps);
+                else qk.template item<true>(tp, fp, v, lane, ps);
+            } else {
+                qk.skip(lane, ps);
+            }
+            if (lane == 0) reinterpret_cast<int *>(ps)[C::PITEM] = it;
+            mbar_arrive(&p_full[pw * C::DP + slot]);
+        }
+    } else {
+        pv.init();
+        for (int k = 0;; ++k) {
+            const int slot = k % C::DP;
+            const float *ps = pring + (pw * C::DP + slot) * C::PSLOT;
+            // p_full implies the QK warp saw the stage ready, hence landed
+            if (!mbar_wait_bounded(&p_full[pw * C::DP + slot], (k / C::DP) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            const int it = reinterpret_cast<const int *>(ps)[C::PITEM];
+            if (it < 0) break;
+            float4 pp[C::TPI / 2];
+#pragma unroll
+            for (int h = 0; h < C::TPI / 2; ++h) pp[h] = lds128f(ps + lane * 2 * C::TPI + 4 * h);
+            const float2 al = make_float2(ps[C::PA + 2 * (lane & 3)], ps[C::PA + 2 * (lane & 3) + 1]);
+            mbar_arrive(&p_empty[pw * C::DP + slot]);
+            const int st = it / C::ITEMS_PER_STAGE, si = st % C::NS, within = it % C::ITEMS_PER_STAGE;
+            const int tok = t0 + it * C::TPI * TILE;
+            int v[C::TPI];
+#pragma unroll
+            for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
+            const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
+            const bool ok = stage_ok[si] != 0;
+            if (v[C::TPI - 1] == TILE) pv.template item<false>(tp, v, ok, lane, pp, al);
+            else pv.template item<true>(tp, v, ok, lane, pp, al);
+            mbar_arrive(&empty[si]);
+        }
+    }
+
+    // ---- CTA merge: QK warps report (m, l); PV warps write o scaled to the CTA
+    // max into their own buffer; the merge threads sum the buffers into the
+    // partial -----------------------------------------------------------------
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));               // every consumer is done with the ring
+    float *obuf = reinterpret_cast<float *>(smem);            // [NQK][8][OSTRIDE]
+    float *m_s = obuf + C::NQK * 8 * C::OSTRIDE;              // [NQK][8]
+    float *l_s = m_s + C::NQK * 8;                            // [NQK][8]
+    if (is_qk) {
+        float lr = qk.l_run;
+        lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+        lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+        if ((lane & 3) == 0) {
+            m_s[pw * 8 + (lane >> 2)] = qk.m_run;
+            l_s[pw * 8 + (lane >> 2)] = lr;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    if (!is_qk) {
+        const int t = lane & 3;
+        float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) {
+            M0 = fmaxf(M0, m_s[w * 8 + 2 * t]);
+            M1 = fmaxf(M1, m_s[w * 8 + 2 * t + 1]);
+        }
+        const float m0 = m_s[pw * 8 + 2 * t], m1 = m_s[pw * 8 + 2 * t + 1];
+        const float sc0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0), sc1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
+        pv.store_scaled(obuf + pw * 8 * C::OSTRIDE, sc0, sc1, lane);
+    } else if (pw == 0 && lane < 8) {
+        const int h = lane;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) M = fmaxf(M, m_s[w * 8 + h]);
+        float Lh = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) {
+            const float mw = m_s[w * 8 + h];
+            if (mw != -INFINITY) Lh += l_s[w * 8 + h] * exp2f(mw - M);
+        }
+        wsu[G * D + h] = M;
+        wsu[G * D + 8 + h] = Lh;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCT));
+    for (int i = threadIdx.x; i < G * D; i += NCT) {
+        const float *b = obuf + (i >> 8) * C::OSTRIDE + (i & 255);
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::NQK; ++w) acc += b[w * 8 * C::OSTRIDE];
+        wsu[i] = acc;
+    }
+    publish_unit<FUSED, NCT>(A, seq, kvh, n_units, &s_last, smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -1512,7 +1507,7 @@ template <int FMT, int GT, bool FUSED>
 __global__ void __launch_bounds__(AluCfg<FMT>::NTHREADS, 1) decode_alu_kernel(const DecodeArgs A) {
     using L = TileLayout<FMT>;
     using C = AluCfg<FMT>;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     grid_dependency_wait();
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *empty = full + C::NS;
@@ -1635,13 +1630,13 @@ cudaError_t launch_decode_kernel(int smem_bytes, int threads, const DecodeArgs &
 template <int FMT, bool FUSED>
 cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s) {
     if (tc) {
-        using C = UmCfg<FMT>;
+        using C = TcCfg<FMT>;
         if constexpr (FUSED) {
             if (a.k_new)
-                return launch_decode_kernel<decode_umma_kernel<FMT, true, true>>(C::TOTAL, C::NTHREADS, a, n_units,
-                                                                                 true, s);
+                return launch_decode_kernel<decode_tc_kernel<FMT, true, true>>(C::TOTAL, C::NTHREADS, a, n_units, true,
+                                                                               s);
         }
-        return launch_decode_kernel<decode_umma_kernel<FMT, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+        return launch_decode_kernel<decode_tc_kernel<FMT, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
     }
     using C = AluCfg<FMT>;
     switch (a.G) {

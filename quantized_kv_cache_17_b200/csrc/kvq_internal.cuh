@@ -17,8 +17,7 @@ constexpr int D = 256;            // head_dim
 constexpr int PAGE = 256;         // tokens per page
 constexpr int TILE = 8;           // tokens per tile
 constexpr int TILES_PER_PAGE = PAGE / TILE;
-constexpr int STEP_TOKENS = 64;   // tokens of one bulk copy of the decode's data path (8 tiles)
-constexpr int PLAN_TOKENS = 128;  // granularity of the split plan (one stage of the tensor-core decode)
+constexpr int STEP_TOKENS = 64;   // granularity of the split plan (one pipeline stage)
 constexpr int PLAN_HEADER = 8;
 constexpr int PLAN_MAGIC = 0x4B565131;  // "KVQ1"
 constexpr int WS_TAIL = 16;       // m[8], l[8] after o[G][256] in one workspace unit
@@ -34,23 +33,23 @@ constexpr int WS_TAIL = 16;       // m[8], l[8] after o[G][256] in one workspace
 //
 // Formats: INT8 = (K I8, V I8); Q4_0 = (K Q4, V Q4); K8V4 = (K I8, V Q4).
 //
-// Code arrangement inside a tile (r = token in tile 0..7), chosen for the
-// tensor-core decode: a thread that owns a token reads its K codes, and a
-// thread that owns a dimension reads its V codes, in 16-byte (K) or 4 / 8-byte
-// (V) shared-memory loads without bank conflicts.
+// Code arrangement inside a tile (r = token in tile 0..7).  Each is the
+// register-fragment order of mma.sync.m16n8k16 so that lane (g = lane/4,
+// t = lane%4) finds its operands in 16-byte words at lane*16 of 512-byte rows:
 //
-//  K side, Q4: token r owns the 128 bytes at 128r.  Block b (dims 32b ..
-//      32b+31) is the 16-byte chunk at 16 (b ^ r) of them; its word i holds
-//      dims 32b + 8i .. +7, dim 32b + 8i + 2(n&3) + (n>>2) in nibble n, so that
-//      masking the word with 0x000F000F, 0x00F000F0 and the same after a shift
-//      by 8 gives the dim pairs (0,1), (2,3), (4,5), (6,7) in fp16 halves.
-//  K side, I8: token r owns the 256 bytes at 256r; dims 16j .. 16j+15 are the
-//      16-byte chunk at 16 (j ^ r) of them, in dim order.
-//  V side, Q4: word d (at 4d) holds dim d of the tile's 8 tokens, token
-//      2(n&3) + (n>>2) in nibble n (the same pairing as on the K side).
-//  V side, I8: dim d owns the 8 bytes at 8d, token r in byte r.
-//  Scales (fp16): token r's block scales are contiguous, block b at 2b:
-//      Q4 at 16r (8 blocks), I8 at 8r (4 groups of 64).
+//  K side, Q4: 32-bit word W(r, b, j) (block b = 32 dims, j 0..3) at
+//      (b>>2)*512 + (r*4 + j)*16 + (b&3)*4; nibble n holds dim
+//      32b + 8(n&3) + (n>>2) + 2j.
+//  V side, Q4: word W(p, b, g) (token pair p: tokens 2p, 2p+1; g 0..7) at
+//      (b>>2)*512 + (g*4 + p)*16 + (b&3)*4; nibble n holds token 2p + (n>>2),
+//      dim 32b + g + 8(n&3).
+//  K side, I8: word W(r, s, j) (k-step s = 16 dims) at
+//      (s>>2)*512 + (r*4 + j)*16 + (s&3)*4; byte n holds dim 16s + 2j + {0,1,8,9}[n].
+//  V side, I8: word W(p, m, g) (m-tile m = 16 dims) at
+//      (m>>2)*512 + (g*4 + p)*16 + (m&3)*4; byte n holds token 2p + (n&1),
+//      dim 16m + g + 8(n>>1).
+//  Scales (fp16): Q4 token r, block b at (r>>1)*32 + b*4 + (r&1)*2;
+//                 I8 token r, group q at (r>>1)*16 + q*4 + (r&1)*2.
 // int8 codes are stored as two's complement bytes.
 // ---------------------------------------------------------------------------
 enum Part : int { PART_Q4 = 0, PART_I8 = 1 };
@@ -257,99 +256,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-
-// ---------------------------------------------------------------------------
-// tcgen05 (fifth-generation tensor core) helpers.  Tensor memory (TMEM) is 128
-// lanes x 512 columns of 32 bits per SM; an address is (lane << 16) | column,
-// and a warp reaches only the 32 lanes 32 (warp % 4) .. 32 (warp % 4) + 31.
-// ---------------------------------------------------------------------------
-// Allocate ncols columns (a power of two >= 32) for this CTA; the whole warp
-// executes it and the base address lands in *dst (shared memory).
-__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// Order tcgen05 operations against thread synchronisation (barriers,
-// mbarriers): "before" on the signalling side, "after" on the waiting side.
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Arrive once on bar when every tcgen05.mma this thread issued so far is complete.
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, no swizzle: 8-row x 16-byte core matrices,
-// lbo / sbo = byte distances between core matrices along the leading / strided
-// dimension (both multiples of 16), version field 1.
-__device__ __forceinline__ uint64_t umma_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-// Instruction descriptor of kind::f16: fp16 A and B, fp32 accumulator, A
-// K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1).
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, int b_mn) {
-    return (1u << 4) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-// D (TMEM) [+]= A (TMEM, 128 lanes x 16 fp16 in 8 columns) x B (shared memory).
-__device__ __forceinline__ void umma_f16_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, bool acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc)
-        : "memory");
-}
-
-// Each lane of the warp moves N consecutive 32-bit columns of its own TMEM
-// lane (lane field of taddr = 32 (warp % 4)).
-template <int N> struct Tmem;
-#define KVQ_R(i) "r"(r[i])
-#define KVQ_W(i) "=r"(r[i])
-template <> struct Tmem<16> {
-    __device__ __forceinline__ static void st(uint32_t ta, const uint32_t (&r)[16]) {
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                     "%15,%16};" ::"r"(ta), KVQ_R(0), KVQ_R(1), KVQ_R(2), KVQ_R(3), KVQ_R(4), KVQ_R(5), KVQ_R(6),
-                     KVQ_R(7), KVQ_R(8), KVQ_R(9), KVQ_R(10), KVQ_R(11), KVQ_R(12), KVQ_R(13), KVQ_R(14), KVQ_R(15)
-                     : "memory");
-    }
-    __device__ __forceinline__ static void ld(uint32_t ta, uint32_t (&r)[16]) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-                     "[%16];"
-                     : KVQ_W(0), KVQ_W(1), KVQ_W(2), KVQ_W(3), KVQ_W(4), KVQ_W(5), KVQ_W(6), KVQ_W(7), KVQ_W(8),
-                       KVQ_W(9), KVQ_W(10), KVQ_W(11), KVQ_W(12), KVQ_W(13), KVQ_W(14), KVQ_W(15)
-                     : "r"(ta)
-                     : "memory");
-    }
-};
-template <> struct Tmem<32> {
-    __device__ __forceinline__ static void st(uint32_t ta, const uint32_t (&r)[32]) {
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                     "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(ta),
-                     KVQ_R(0), KVQ_R(1), KVQ_R(2), KVQ_R(3), KVQ_R(4), KVQ_R(5), KVQ_R(6), KVQ_R(7), KVQ_R(8),
-                     KVQ_R(9), KVQ_R(10), KVQ_R(11), KVQ_R(12), KVQ_R(13), KVQ_R(14), KVQ_R(15), KVQ_R(16),
-                     KVQ_R(17), KVQ_R(18), KVQ_R(19), KVQ_R(20), KVQ_R(21), KVQ_R(22), KVQ_R(23), KVQ_R(24),
-                     KVQ_R(25), KVQ_R(26), KVQ_R(27), KVQ_R(28), KVQ_R(29), KVQ_R(30), KVQ_R(31)
-                     : "memory");
-    }
-    __device__ __forceinline__ static void ld(uint32_t ta, uint32_t (&r)[32]) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-                     "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                     : KVQ_W(0), KVQ_W(1), KVQ_W(2), KVQ_W(3), KVQ_W(4), KVQ_W(5), KVQ_W(6), KVQ_W(7), KVQ_W(8),
-                       KVQ_W(9), KVQ_W(10), KVQ_W(11), KVQ_W(12), KVQ_W(13), KVQ_W(14), KVQ_W(15), KVQ_W(16),
-                       KVQ_W(17), KVQ_W(18), KVQ_W(19), KVQ_W(20), KVQ_W(21), KVQ_W(22), KVQ_W(23), KVQ_W(24),
-                       KVQ_W(25), KVQ_W(26), KVQ_W(27), KVQ_W(28), KVQ_W(29), KVQ_W(30), KVQ_W(31)
-                     : "r"(ta)
-                     : "memory");
-    }
-};
-#undef KVQ_R
-#undef KVQ_W
 
 __device__ __forceinline__ void status_or(int32_t *status, uint32_t bits) {
     if (status) atomicOr(reinterpret_cast<unsigned int *>(status), bits);

@@ -31,33 +31,37 @@ def code_map(part: str, side: str):
     off = np.full((8, 256), -1, np.int64)
     sh = np.zeros((8, 256), np.int64)
     if part == Q4 and side == "k":
-        # token r: 128 bytes at 128r; block b in the 16-byte chunk at 16 (b ^ r);
-        # word i of it: dims 32b + 8i + 2(n&3) + (n>>2) in nibble n
         for r in range(8):
             for b in range(8):
-                for i in range(4):
+                for j in range(4):
                     for n in range(8):
-                        d = 32 * b + 8 * i + 2 * (n & 3) + (n >> 2)
-                        off[r, d] = 128 * r + 16 * (b ^ r) + 4 * i + (n >> 1)
+                        d = 32 * b + 8 * (n & 3) + (n >> 2) + 2 * j
+                        off[r, d] = (b >> 2) * 512 + (r * 4 + j) * 16 + (b & 3) * 4 + (n >> 1)
                         sh[r, d] = 4 * (n & 1)
     elif part == Q4 and side == "v":
-        # one 32-bit word per dim: token r in nibble 4(r&1) + (r>>1)
-        for r in range(8):
-            n = 4 * (r & 1) + (r >> 1)
-            for d in range(256):
-                off[r, d] = 4 * d + (n >> 1)
-                sh[r, d] = 4 * (n & 1)
+        for p in range(4):
+            for b in range(8):
+                for g in range(8):
+                    for n in range(8):
+                        r = 2 * p + (n >> 2)
+                        d = 32 * b + g + 8 * (n & 3)
+                        off[r, d] = (b >> 2) * 512 + (g * 4 + p) * 16 + (b & 3) * 4 + (n >> 1)
+                        sh[r, d] = 4 * (n & 1)
     elif part == I8 and side == "k":
-        # token r: 256 bytes at 256r; dims 16j .. 16j+15 in the chunk at 16 (j ^ r)
         for r in range(8):
-            for j in range(16):
-                for e in range(16):
-                    off[r, 16 * j + e] = 256 * r + 16 * (j ^ r) + e
+            for s in range(16):
+                for j in range(4):
+                    for n, dd in enumerate((0, 1, 8, 9)):
+                        d = 16 * s + 2 * j + dd
+                        off[r, d] = (s >> 2) * 512 + (r * 4 + j) * 16 + (s & 3) * 4 + n
     elif part == I8 and side == "v":
-        # 8 bytes per dim: token r in byte r
-        for r in range(8):
-            for d in range(256):
-                off[r, d] = 8 * d + r
+        for p in range(4):
+            for m in range(16):
+                for g in range(8):
+                    for n in range(4):
+                        r = 2 * p + (n & 1)
+                        d = 16 * m + g + 8 * (n >> 1)
+                        off[r, d] = (m >> 2) * 512 + (g * 4 + p) * 16 + (m & 3) * 4 + n
     else:
         raise ValueError((part, side))
     assert (off >= 0).all()
@@ -68,10 +72,11 @@ def code_map(part: str, side: str):
 def scale_map(part: str):
     """byte offset of the fp16 scale of (token r, block q): [8, n_scales]."""
     ns = N_SCALES[part]
+    stride = 32 if part == Q4 else 16
     off = np.zeros((8, ns), np.int64)
     for r in range(8):
         for q in range(ns):
-            off[r, q] = 2 * ns * r + 2 * q
+            off[r, q] = (r >> 1) * stride + q * 4 + (r & 1) * 2
     return off
 
 

@@ -183,7 +183,7 @@ def test_decode_bad_plan_reports_status():
     w = small("int8", 4, 1, [300])
     dw = kdev.build_pool(w, prefill_last=True)
     plan, info = kvq.decode_plan(dw.pool.desc, dw.seq_lens, dw.page_table.shape[1], 0)
-    plan[8 + 2] = 32            # unit start not on a plan step (128 tokens)
+    plan[8 + 2] = 32            # unit start not on a 64-token step
     plan_d = torch.from_numpy(plan).cuda()
     ws = torch.empty(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")

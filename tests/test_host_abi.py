@@ -87,7 +87,7 @@ def _check_plan(plan, info, seq_lens, n_kv, n_ctas):
             assert (us[:, 0] == b).all() and (us[:, 1] == g).all()
             assert us[0, 2] == 0 and us[-1, 3] == T
             assert (us[1:, 2] == us[:-1, 3]).all()          # contiguous, no overlap, no gap
-            assert (us[:, 2] % 128 == 0).all() and (us[:, 3] > us[:, 2]).all()
+            assert (us[:, 2] % 64 == 0).all() and (us[:, 3] > us[:, 2]).all()
             assert ((us[:, 3] - us[:, 2]) <= info.chunk_tokens).all()
     G = plan[4]
     counters = (len(seq_lens) * n_kv * 4 + 15) // 16 * 16
@@ -109,7 +109,7 @@ def test_decode_plan_balance_full_window():
     units = plan[8:8 + 4 * info.n_units].reshape(-1, 4)
     sizes = units[:, 3] - units[:, 2]
     assert info.n_units == 148
-    assert sizes.max() - sizes.min() <= 128
+    assert sizes.max() - sizes.min() <= 64
 
 
 def test_validation_errors_without_a_gpu():
