@@ -117,19 +117,43 @@ __device__ __forceinline__ void sts128(void *p, uint4 v) {
                  : "memory");
 }
 
+// Warpgroup register budgets (every warp of the warpgroup executes the same
+// instruction; .inc waits until .dec has returned enough registers).
+template <int N> __device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core kernel: configuration
 // ---------------------------------------------------------------------------
-#ifndef KVQ_QK_WARPS
-#define KVQ_QK_WARPS 7       // QK warps per CTA (and as many PV warps)
-#endif
-
+// Warp roles, in warpgroups of four: NQK QK warps, NQK PV warps, then one
+// producer warpgroup: the copy warp and N_SCALE scale warps.  Each SM
+// sub-partition (warp index mod 4) then holds two pairs and one producer; the
+// scale work is split by ring slot so that no sub-partition carries all of it
+// (a sub-partition whose producer did all the conversions ran its pairs about
+// a quarter slower, and every pair waits for the slowest through the ring).  The
+// launch gives every thread REG_LAUNCH registers; at the start the producer
+// warpgroup gives registers back (setmaxnreg.dec) and the QK and PV
+// warpgroups take them (setmaxnreg.inc), so that eight pairs fit on the SM:
+// two per SM sub-partition, where seven pairs loaded two of the four with an
+// extra pair's work.
 template <int FMT> struct TcCfg {
     using L = TileLayout<FMT>;
-    static constexpr int NQK = KVQ_QK_WARPS;
-    static constexpr int SCALE_WARP = 2 * NQK;
-    static constexpr int COPY_WARP = 2 * NQK + 1;
-    static constexpr int NTHREADS = (2 * NQK + 2) * 32;
+    static constexpr int NQK = 8;
+    static constexpr int COPY_WARP = 2 * NQK;
+    static constexpr int SCALE_WARP = 2 * NQK + 1;               // the first of N_SCALE
+    static constexpr int N_SCALE = 3;
+    static constexpr int NTHREADS = (2 * NQK + 4) * 32;
+    static constexpr int REG_LAUNCH = 65536 / NTHREADS / 8 * 8;     // 96
+    static constexpr int REG_COMPUTE = 112, REG_PROD = 32;
+    static_assert(NQK % 4 == 0, "QK and PV warps fill whole warpgroups");
+    // the warpgroups' budgets after the split add up to what the launch holds
+    static_assert(2 * NQK * REG_COMPUTE + 4 * REG_PROD <= NTHREADS / 32 * REG_LAUNCH,
+                  "register split exceeds the launch's registers");
+    static_assert(SCALE_WARP + N_SCALE == NTHREADS / 32, "producer warpgroup: copy warp + scale warps");
     static constexpr int TPI = FMT == KVQ_INT8 ? 2 : 4;         // tiles per work item (measured best)
     static constexpr int ITEMS_PER_STAGE = 8 / TPI;
     static constexpr int STAGE_BYTES = 8 * L::BYTES;
@@ -153,7 +177,9 @@ template <int FMT> struct TcCfg {
     static constexpr int POFF = SFOFF + NS * SF_STAGE_BYTES;
     // the QK -> PV rings; before the loop, the group's query (KVQ_MAX_GROUP heads)
     static constexpr int PRING_FLOATS = NQK * DP * PSLOT > KVQ_MAX_GROUP * D ? NQK * DP * PSLOT : KVQ_MAX_GROUP * D;
-    static constexpr int BAR_OFF = POFF + PRING_FLOATS * 4;
+    // the group's query as MMA A fragments: [16 k-steps][32 lanes] x 16 bytes
+    static constexpr int QOFF = POFF + PRING_FLOATS * 4;
+    static constexpr int BAR_OFF = QOFF + 16 * 32 * 16;
     // full, ready, empty [NS]; p_full, p_empty [NQK * DP]; stage_ok [NS]; then,
     // for a decode step, the newest token's codes and scales (5 words per lane)
     static constexpr int TKV_OFF = (BAR_OFF + (3 * NS + 2 * NQK * DP) * 8 + NS * 4 + 15) & ~15;
@@ -247,7 +273,7 @@ template <int FMT> struct QkWarp {
     using L = TileLayout<FMT>;
     using C = TcCfg<FMT>;
     using K = QkCodes<FMT>;
-    uint4 qa[16];          // A fragments of the 16 k-steps (scaled by 2^kq)
+    const uint8_t *qf;     // A fragments of the 16 k-steps (scaled by 2^kq), shared by the QK warps
     uint32_t qb_hi, qb_lo; // A fragment of the offset MMA: -OFF 2^-KBS Q[2t], Q[2t+1] of head g, hi / lo rows
     float inv_sb;          // 2^-kb
     float m_run, l_run;    // head g (the four lanes of a group agree)
@@ -257,8 +283,13 @@ template <int FMT> struct QkWarp {
     // Fragments of head g (rows g: fp16 hi, g+8: fp16 lo), k-step ks: dims
     // 16ks + 2t, +1 (x, y) and 16ks + 2t + 8, +9 (z, w).  For 4-bit keys the
     // second pair is divided by 16, matching its codes' 16 code * 2^-24.
-    __device__ __forceinline__ void init(const float *qg, int G, int lane) {
+    __device__ __forceinline__ uint4 qa(int ks, int lane) const { return lds128(qf + (ks * 32 + lane) * 16); }
+
+    // Every QK warp computes the fragments (and its own offset fragment);
+    // `writer` stores them to q_frag.
+    __device__ __forceinline__ void init(const float *qg, int G, int lane, uint8_t *q_frag, bool writer) {
         const int g = lane >> 2, t = lane & 3;
+        qf = q_frag;
         float mx = 0.f;
         if (g < G) {
 #pragma unroll
@@ -289,7 +320,7 @@ template <int FMT> struct QkWarp {
             uint4 f;
             split_pair(x[0], x[1], f.x, f.y);
             split_pair(x[2], x[3], f.z, f.w);
-            qa[ks] = f;
+            if (writer) sts128(q_frag + (ks * 32 + lane) * 16, f);
             const float2 h0 = __half22float2(u32_as_h2(f.x)), l0 = __half22float2(u32_as_h2(f.y));
             const float2 h1 = __half22float2(u32_as_h2(f.z)), l1 = __half22float2(u32_as_h2(f.w));
             const float r = ((h0.x + l0.x) + (h0.y + l0.y)) + M_HI * ((h1.x + l1.x) + (h1.y + l1.y));
@@ -357,10 +388,11 @@ template <int FMT> struct QkWarp {
                     const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
                     const uint32_t wA2 = wA >> 8, wB2 = wB >> 8;
                     float a[4], c[4];
-                    mma_z(a, qa[2 * b], wA & 0x000F000Fu, wA & 0x00F000F0u);
-                    mma_z(c, qa[2 * b], wB & 0x000F000Fu, wB & 0x00F000F0u);
-                    mma_acc(a, qa[2 * b + 1], wA2 & 0x000F000Fu, wA2 & 0x00F000F0u);
-                    mma_acc(c, qa[2 * b + 1], wB2 & 0x000F000Fu, wB2 & 0x00F000F0u);
+                    const uint4 q0 = qa(2 * b, lane), q1 = qa(2 * b + 1, lane);
+                    mma_z(a, q0, wA & 0x000F000Fu, wA & 0x00F000F0u);
+                    mma_z(c, q0, wB & 0x000F000Fu, wB & 0x00F000F0u);
+                    mma_acc(a, q1, wA2 & 0x000F000Fu, wA2 & 0x00F000F0u);
+                    mma_acc(c, q1, wB2 & 0x000F000Fu, wB2 & 0x00F000F0u);
                     const float2 da = f2_at(dA0, dA1, bb), db = f2_at(dB0, dB1, bb);
                     s[0] = fmaf(a[0] + a[2], da.x, s[0]);
                     s[1] = fmaf(a[1] + a[3], da.y, s[1]);
@@ -381,12 +413,13 @@ template <int FMT> struct QkWarp {
                     const uint32_t wA = u4_at(kA, j) ^ 0x80808080u, wB = u4_at(kB, j) ^ 0x80808080u;
                     const uint32_t a0 = __byte_perm(wA, 0u, 0x4140u), a1 = __byte_perm(wA, 0u, 0x4342u);
                     const uint32_t b0 = __byte_perm(wB, 0u, 0x4140u), b1 = __byte_perm(wB, 0u, 0x4342u);
+                    const uint4 qj = qa(4 * q + j, lane);
                     if (j == 0) {
-                        mma_z(a, qa[4 * q], a0, a1);
-                        mma_z(c, qa[4 * q], b0, b1);
+                        mma_z(a, qj, a0, a1);
+                        mma_z(c, qj, b0, b1);
                     } else {
-                        mma_acc(a, qa[4 * q + j], a0, a1);
-                        mma_acc(c, qa[4 * q + j], b0, b1);
+                        mma_acc(a, qj, a0, a1);
+                        mma_acc(c, qj, b0, b1);
                     }
                 }
                 const float2 da = f2_at(dA0, dA1, q), db = f2_at(dB0, dB1, q);
@@ -1114,14 +1147,19 @@ __device__ __forceinline__ void copy_loop(const DecodeArgs &A, uint8_t *smem, ui
         }
         const int slot = __shfl_sync(0xffffffffu, my_slot, rel & 31);
         hook(i, lane);                 // whole warp, before step i is requested
+        // the whole warp waits for the free stage (a warp whose lane 0 waits
+        // alone while the rest sit at the warp barrier slowed the other warps
+        // of its SM sub-partition)
+        bool free_stage = stop || i < NS || mbar_wait_bounded(&empty[i % NS], ((i / NS) - 1) & 1, WAIT_LIMIT_NS);
+        free_stage = __all_sync(0xffffffffu, free_stage);
+        if (!free_stage) {                       // a stage never came free: issue nothing more
+            if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+            stop = true;
+        }
         if (lane == 0 && !stop) {
             ++issued;
             const int si = i % NS;
-            if (i >= NS && !mbar_wait_bounded(&empty[si], ((i / NS) - 1) & 1, WAIT_LIMIT_NS)) {
-                status_or(A.status, KVQ_STATUS_TIMEOUT);
-                stop = true;
-                --issued;
-            } else if (slot < 0 || slot >= A.geo.n_pages) {
+            if (slot < 0 || slot >= A.geo.n_pages) {
                 status_or(A.status, KVQ_STATUS_BAD_SLOT);
                 stage_ok[si] = 0;
                 mbar_arrive(&full[si]);
@@ -1326,29 +1364,46 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
     // decode step: the last CTA of the group appends the group's newest token
     const bool appends = STEP && u == A.plan[PLAN_HEADER + 4 * n_units + seq * A.geo.n_kv_heads + kvh + 1] - 1;
 
-    if (warp == C::COPY_WARP) {
-        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
-        return;
-    }
-    if (warp == C::SCALE_WARP) {
+    if (warp >= 2 * C::NQK) {                   // the producer warpgroup
+        setmaxnreg_dec<C::REG_PROD>();
+        if (warp == C::COPY_WARP)
+            copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, seq, kvh, t0, n_steps, lane);
+        if (warp < C::SCALE_WARP) return;
+        // scale warp c owns the ring slots si with si % N_SCALE == c, so each
+        // slot's phases are awaited by one warp, in order.  The stages still
+        // become ready in order: a QK warp waits on the ready barrier of a stage
+        // up to NQK items past its last one, and a barrier two phases behind
+        // would answer that wait with an older phase of the same parity.  So a
+        // scale warp converts as soon as its stage lands, but announces it only
+        // after the previous stage's announcement.
+        const int c = warp - C::SCALE_WARP;
         uint32_t *stash = reinterpret_cast<uint32_t *>(smem + C::TKV_OFF);
-        if (appends) step_encode_token<FMT>(A, seq, kvh, t1 - 1, stash, lane);
+        const bool encodes = appends && ((n_steps - 1) % C::NS) % C::N_SCALE == c;   // owns the newest token's stage
+        if (encodes) step_encode_token<FMT>(A, seq, kvh, t1 - 1, stash, lane);
         for (int i = 0; i < n_steps; ++i) {
             const int si = i % C::NS;
+            if (si % C::N_SCALE != c) continue;
             if (!mbar_wait_bounded(&full[si], (i / C::NS) & 1, WAIT_LIMIT_NS)) {
                 if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
                 break;
             }
-            if (appends && i == n_steps - 1 && stage_ok[si])    // the stage that holds the newest token
+            if (encodes && i == n_steps - 1 && stage_ok[si])    // the stage that holds the newest token
                 step_patch_stage<FMT>(t1 - 1, stash, smem + si * C::STAGE_BYTES, lane);
             if (stage_ok[si])
                 convert_stage_scales<FMT>(smem + si * C::STAGE_BYTES,
                                           reinterpret_cast<float *>(smem + C::SFOFF + si * C::SF_STAGE_BYTES), lane);
+            // (the ready barrier of stage i - 1 is at most one phase behind,
+            // since stage i's copy waited for the consumers of stage i - NS)
+            if (i > 0 && !mbar_wait_bounded(&ready[(i - 1) % C::NS], ((i - 1) / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
             __syncwarp();
             mbar_arrive(&ready[si]);
         }
         return;
     }
+    setmaxnreg_inc<C::REG_COMPUTE>();          // QK and PV warpgroups
 
     float *pring = reinterpret_cast<float *>(smem + C::POFF);
     constexpr int NCT = 2 * C::NQK * 32;       // merge threads: QK + PV warps
@@ -1368,7 +1423,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         // rotates the raw query on the way, as q_rotate would.
         step_stage_query<STEP && Fmt<FMT>::KROT>(qg, pring, G, pw, C::NQK, lane);
         asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
-        qk.init(pring, G, lane);
+        qk.init(pring, G, lane, smem + C::QOFF, pw == 0);
         asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
         for (int k = 0;; ++k) {
             const int slot = k % C::DP;
@@ -1598,10 +1653,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 // shared-memory limit and counts how many of its CTAs fit on the device at
 // once (for this very kernel, so the cooperative decision matches what is
 // launched); both happen once per (kernel, device) under a lock, so threads
-// may launch concurrently.
+// may launch concurrently.  A kernel that moves registers between warpgroups
+// (regs > 0) is launched only if it was built with exactly that many
+// registers per thread: with fewer, its setmaxnreg.inc could never be met.
 template <auto KERNEL>
 cudaError_t launch_decode_kernel(int smem_bytes, int threads, const DecodeArgs &a, int n_units, bool fused,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, int regs = 0) {
     static std::mutex mu;
     static int cap[64];                  // resident CTAs per device ordinal; 0 = not yet known
     int dev = 0;
@@ -1610,6 +1667,12 @@ cudaError_t launch_decode_kernel(int smem_bytes, int threads, const DecodeArgs &
     {
         std::lock_guard<std::mutex> lock(mu);
         if (cap[dev] == 0) {
+            if (regs > 0) {
+                cudaFuncAttributes fa;
+                cudaError_t e = cudaFuncGetAttributes(&fa, KERNEL);
+                if (e != cudaSuccess) return e;
+                if (fa.numRegs != regs) return cudaErrorInvalidConfiguration;
+            }
             cudaError_t e = cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
             if (e != cudaSuccess) return e;
             int sms = 0, per_sm = 0;
@@ -1634,9 +1697,10 @@ cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s
         if constexpr (FUSED) {
             if (a.k_new)
                 return launch_decode_kernel<decode_tc_kernel<FMT, true, true>>(C::TOTAL, C::NTHREADS, a, n_units, true,
-                                                                               s);
+                                                                               s, C::REG_LAUNCH);
         }
-        return launch_decode_kernel<decode_tc_kernel<FMT, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+        return launch_decode_kernel<decode_tc_kernel<FMT, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s,
+                                                                  C::REG_LAUNCH);
     }
     using C = AluCfg<FMT>;
     switch (a.G) {
