@@ -145,26 +145,68 @@ def weak_scaling_gbs(world: int, bytes_per_rank_step: float, ms_per_step: float)
     return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
 
 
-def cpu_oracle_rate(fmt: str, G: int, groups, budget_s: float):
-    """Time the oracle (single thread, as it stands) on (layer, KV head) groups;
-    `groups` yields ((kc, ks, vc, vs), qp) and only the oracle calls are timed.
-    Returns (KV GB/s, token-kvheads/s, seconds, groups done)."""
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_parallel(fmt: str, groups, threads: int):
+    """The oracle (as it stands) over whole (layer, KV head) groups on `threads`
+    host threads: every group's token range is cut into chunks, each chunk is
+    one oracle partial (the oracle's own split form, ctypes releases the GIL),
+    and each group's partials are merged with the oracle's merge.  `groups` is
+    a list of ((kc, ks, vc, vs), qp).  Returns (seconds, tokens, bytes)."""
+    from concurrent.futures import ThreadPoolExecutor
     import oracle
-    dt = 0.0
-    done_bytes = 0
-    done_tok = 0
-    n = 0
     per_tok = oracle.format_bytes_per_token_head(fmt)
-    for (kc, ks, vc, vs), qp in groups:
-        t0 = time.perf_counter()
-        oracle.attn_decode(fmt, qp, kc, ks, vc, vs)
-        dt += time.perf_counter() - t0
-        done_tok += kc.shape[0]
-        done_bytes += kc.shape[0] * per_tok
-        n += 1
-        if dt > budget_s:
-            break
-    return done_bytes / dt / 1e9, done_tok / dt, dt, n
+    n_chunks = max(1, -(-threads // len(groups)))
+    tasks = []
+    for gi, (codes, qp) in enumerate(groups):
+        T = codes[0].shape[0]
+        for c in range(n_chunks):
+            t0, t1 = c * T // n_chunks, (c + 1) * T // n_chunks
+            if t1 > t0:
+                tasks.append((gi, t0, t1))
+
+    def run(task):
+        gi, t0, t1 = task
+        codes, qp = groups[gi]
+        return gi, oracle.attn_partial(fmt, qp, t0, t1, *codes)
+
+    t_start = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        parts = list(ex.map(run, tasks))
+    merged = {}
+    for gi, part in parts:
+        merged[gi] = part if gi not in merged else oracle.merge_partials(merged[gi], part)
+    for gi, (m, l, o) in merged.items():
+        oracle.finish(fmt, l, o)
+    dt = time.perf_counter() - t_start
+    tokens = sum(c[0].shape[0] for c, _ in groups)
+    return dt, tokens, tokens * per_tok
+
+
+def cpu_append_us(fmt: str, n_kv: int, layers: int, k_rows: np.ndarray, v_rows: np.ndarray, reps: int = 20):
+    """The oracle's kv_append of one decode step (one token per KV head and
+    layer), single thread, in microseconds per step."""
+    import oracle
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        for _l in range(layers):
+            oracle.append_rows(fmt, k_rows[:n_kv], v_rows[:n_kv])
+    return (time.perf_counter() - t0) / reps * 1e6
 
 
 def run_reference(args):
@@ -182,27 +224,100 @@ def run_reference(args):
     codes = oracle.append_rows(w.fmt, k, v)
     qp = oracle.q_prepare(w.fmt, w.q_row(layer, b)[g * w.group:(g + 1) * w.group])
     per_tok = oracle.format_bytes_per_token_head(w.fmt)
+    cores = host_cores()
+    groups = [(codes, qp)]
     for _ in range(args.warmup):
-        oracle.attn_decode(w.fmt, qp, *codes)
+        cpu_oracle_parallel(w.fmt, groups, cores)
     times = []
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle.attn_decode(w.fmt, qp, *codes)
-        times.append(time.perf_counter() - t0)
+        times.append(cpu_oracle_parallel(w.fmt, groups, cores)[0])
     dt = sum(times) / len(times)
     gbs = T_sample * per_tok / dt / 1e9
-    sample = (f"oracle fp64 attention of one (layer, KV head) group ({w.group} query heads) over "
-              f"{T_sample} tokens of {w.name}, codes from the oracle's own append; single thread")
+    sample = (f"oracle fp64 attention of one (layer, KV head) group ({w.group} query heads) over the first "
+              f"{T_sample} tokens of {w.name} (codes from the oracle's own append), cut into token chunks run "
+              f"on {cores} threads ({cpu_model()}) and merged with the oracle's own merge")
     line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "format": w.fmt, "seq_lens": w.seq_lens, "layers": w.n_layers,
                        "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 256},
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "cpu_model": cpu_model(), "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------------------
+OTHER_WORKLOADS = ("qwen27b_int8_32k", "flashnext_k8v4_128k", "ragged4_q4_0", "ragged4_k8v4")
+
+
+def measure_workload(name: str, layers: int, steps: int, warmup: int, peak: float, uuid: str):
+    """One decode step per layer (paged_decode_step, the bench's timed kernel)
+    of workload `name` restricted to its first `layers` layers, captured as a
+    CUDA graph and timed with CUDA events over `steps` replays, with the SM
+    clocks sampled meanwhile.  The pool of `layers` layers is larger than L2
+    for every workload, so no flush is needed.  Returns a sub-record."""
+    import torch
+    import kvq_inputs
+    import quantized_kv_cache_17_b200 as kvq
+    from kvq_inputs import device as kdev
+    w0 = kvq_inputs.workload(name)
+    w = kvq_inputs.scaled(w0, w0.seq_lens, n_layers=min(layers, w0.n_layers), name=w0.name)
+    L = w.n_layers
+    dw = kdev.build_pool(w, extra_slots=0)
+    q, k_new, v_new, pos = kdev.step_inputs(w, list(range(L)))
+    plan, info = kvq.decode_plan(dw.pool.desc, w.seq_lens, dw.page_table.shape[1], 0)
+    plan_d = torch.from_numpy(plan).cuda()
+    ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    out_bf = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+    out_f = torch.empty((L, w.batch, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    layout = kvq.pool_layout(dw.pool.desc)
+    kv_bytes_layer = sum(w.seq_lens) * w.n_kv_heads * layout.bytes_per_token_head
+
+    def step():
+        for l in range(L):
+            kvq.paged_decode_step(dw.pool, l, q[l], k_new[l], v_new[l], dw.page_table, plan_d, info, ws, out_bf[l],
+                                  out_f[l], status)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"kernel status {status.item()} on {name}"
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            step()
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    n_rep = max(steps, 2)
+    for _ in range(n_rep):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    assert int(status.item()) == 0, f"kernel status {status.item()} on {name}"
+    us_layer = a.elapsed_time(b) * 1e3 / (n_rep * L)
+    gbs = kv_bytes_layer / (us_layer * 1e-6) / 1e9
+    del g
+    rec = {"workload": name, "format": w.fmt, "seq_lens": w.seq_lens, "layers_timed": L,
+           "us_per_layer_step": round(us_layer, 3), "kv_bytes_per_layer": kv_bytes_layer,
+           "gbs": round(gbs, 2), "frac": round(gbs / peak, 4), "n_units": info.n_units, "clocks": clocks}
+    del dw, q, k_new, v_new, ws, out_bf, out_f
+    torch.cuda.empty_cache()
+    return rec
 
 
 # ---------------------------------------------------------------------------
@@ -420,18 +535,37 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         from tests import kvq_layout
-        def groups():
-            b = len(w.seq_lens) - 1
-            for idx in range(min(args.cpu_groups, L * w.n_kv_heads)):
-                lay, g = L - 1 - idx // w.n_kv_heads, idx % w.n_kv_heads   # last layers first
-                codes = kvq_layout.gather_sequence(fmt, dw.pool.buf, layout, lay, g, dw.page_table_host[b],
-                                                   w.seq_lens[b])
-                yield codes, oracle.q_prepare(fmt, q[lay, b, g * w.group:(g + 1) * w.group].cpu().numpy())
-        gbs, tok_rate, dt, n = cpu_oracle_rate(fmt, w.group, groups(), args.cpu_budget)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"oracle fp64 attention of {n} (layer, KV head) groups ({w.group} query heads each) over "
-                         f"{w.seq_lens[-1]} tokens of {w.name}, codes read back from the GPU pool; "
-                         f"single thread, {dt:.1f} s"}
+        b = len(w.seq_lens) - 1
+        cores = host_cores()
+        n_groups = min(args.cpu_groups, L * w.n_kv_heads)
+        groups = []
+        for idx in range(n_groups):
+            lay, g = L - 1 - idx // w.n_kv_heads, idx % w.n_kv_heads          # last layers first
+            codes = kvq_layout.gather_sequence(fmt, dw.pool.buf, layout, lay, g, dw.page_table_host[b], w.seq_lens[b])
+            groups.append((codes, oracle.q_prepare(fmt, q[lay, b, g * w.group:(g + 1) * w.group].cpu().numpy())))
+        dt_all, tok_all, bytes_all = cpu_oracle_parallel(fmt, groups, cores)
+        dt_one, tok_one, bytes_one = cpu_oracle_parallel(fmt, groups[:2], 1)
+        kv_step_seq = w.seq_lens[b] * w.n_kv_heads * L * layout.bytes_per_token_head
+        app_us = cpu_append_us(fmt, w.n_kv_heads, L, k_new[0, b].cpu().numpy(), v_new[0, b].cpu().numpy())
+        cpu = {"value": round(bytes_all / dt_all / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
+               "single_core_gbs": round(bytes_one / dt_one / 1e9, 4),
+               "ms_per_step_all_cores": round(kv_step_seq / (bytes_all / dt_all) * 1e3, 1),
+               "ms_per_step_single_core": round(kv_step_seq / (bytes_one / dt_one) * 1e3, 1),
+               "append_us_per_step": round(app_us, 1),
+               "sample": f"oracle fp64 attention of {n_groups} (layer, KV head) groups ({w.group} query heads each) "
+                         f"over {w.seq_lens[b]} tokens of {w.name}, codes read back from the GPU pool, cut into "
+                         f"token chunks on {cores} threads ({dt_all:.1f} s) and merged with the oracle's merge; "
+                         f"single core: two groups ({dt_one:.1f} s); the ms per 16-layer step figures extrapolate "
+                         f"these rates to all {L * w.n_kv_heads} groups of sequence {b}; append: the oracle's "
+                         f"encode of one token per KV head and layer, single thread"}
+
+    others = None
+    if rank == 0 and world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD and not use_alu \
+            and not args.layers:
+        del dw, q, k_new, v_new, ws, out_bf, out_f, q_rot
+        torch.cuda.empty_cache()
+        others = [measure_workload(n, args.other_layers, args.steps, args.warmup, peak, uuid) for n in OTHER_WORKLOADS]
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -462,7 +596,8 @@ def run_ours(args):
                 "gpu_launches": args.steps * L * launches_per_layer,
                 "launch": "CUDA graph of the 16-layer step",
                 "clocks": clocks,
-                "cpu_baseline": cpu}
+                "cpu_baseline": cpu,
+                "other_workloads": others}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -481,8 +616,9 @@ def main():
     ap.add_argument("--no-fuse", action="store_true", help="separate attn_combine launch")
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-groups", type=int, default=16)
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--cpu-groups", type=int, default=16, help="(layer, KV head) groups in the CPU baseline")
+    ap.add_argument("--no-others", action="store_true", help="skip the sub-records of the other workloads")
+    ap.add_argument("--other-layers", type=int, default=4, help="layers timed per other workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
