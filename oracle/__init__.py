@@ -23,9 +23,15 @@ LIB = os.path.join(HERE, "liboracle_kvq.so")
 # with a deliberately planted mistake) through this variable.
 _OVERRIDE = os.environ.get("KVQ_ORACLE_LIB")
 
-FMT = {"int8": 0, "q4_0": 1, "k8v4": 2}
-# (K is 4-bit, V is 4-bit, K rotated, V rotated) per format
-PARTS = {"int8": (False, False, False, False), "q4_0": (True, True, True, True), "k8v4": (False, True, False, True)}
+FMT = {"int8": 0, "q4_0": 1, "k8v4": 2, "fp8": 3, "nvfp4": 4}
+# How K and V are stored: "i8" (int8, fp16 scale per 64), "q4" (q4_0, fp16
+# scale per 32), "e4m3" (fp8 codes, one fp16 scale), "e2m1" (fp4 codes, an
+# E4M3 scale per 16).
+PART_ID = {"i8": 0, "q4": 1, "e4m3": 2, "e2m1": 3}
+N_SCALES = {"i8": 4, "q4": 8, "e4m3": 1, "e2m1": 16}
+# (K part, V part, K rotated, V rotated) per format
+PARTS = {"int8": ("i8", "i8", False, False), "q4_0": ("q4", "q4", True, True), "k8v4": ("i8", "q4", False, True),
+         "fp8": ("e4m3", "e4m3", False, False), "nvfp4": ("e2m1", "e2m1", False, False)}
 
 _lib = None
 
@@ -55,6 +61,16 @@ def lib():
         L.oracle_fwht256_f64.argtypes = [P, P]
         L.oracle_quant_q4_0.argtypes = [P, P, P]
         L.oracle_quant_int8.argtypes = [P, P, P]
+        L.oracle_quant_fp8.argtypes = [P, P, P]
+        L.oracle_quant_nvfp4.argtypes = [P, P, P]
+        L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_f32.restype = ctypes.c_float
+        L.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_to_f32.restype = ctypes.c_float
+        L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        L.oracle_f32_to_e2m1.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_e2m1.restype = ctypes.c_uint8
         L.oracle_append_rows.argtypes = [ctypes.c_int, ctypes.c_long, P, P, P, P, P, P]
         L.oracle_append_rows.restype = ctypes.c_int
         L.oracle_q_prepare.argtypes = [ctypes.c_int, P, P, ctypes.c_long]
@@ -101,6 +117,26 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return np.array([L.oracle_f32_to_bf16(float(v)) for v in x], np.uint16)
 
 
+def e4m3_to_f32(b: np.ndarray) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_e4m3_to_f32(int(v)) for v in np.asarray(b, np.uint8).ravel()], np.float32)
+
+
+def e2m1_to_f32(c: np.ndarray) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_e2m1_to_f32(int(v)) for v in np.asarray(c, np.uint8).ravel()], np.float32)
+
+
+def f32_to_e4m3(x: np.ndarray) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_f32_to_e4m3(float(v)) for v in np.asarray(x, np.float32).ravel()], np.uint8)
+
+
+def f32_to_e2m1(x: np.ndarray) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_f32_to_e2m1(float(v)) for v in np.asarray(x, np.float32).ravel()], np.uint8)
+
+
 # --- transform / codecs ------------------------------------------------------
 def fwht256_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, np.float32).reshape(-1, 256)
@@ -136,8 +172,36 @@ def quant_int8(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     return c, s
 
 
-def n_scales(is_q4: bool) -> int:
-    return 8 if is_q4 else 4
+def quant_fp8(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """256-vector -> (E4M3 codes uint8[256], fp16 scale bits uint16[1])."""
+    x = np.ascontiguousarray(x, np.float32).reshape(256)
+    c = np.empty(256, np.uint8)
+    s = np.empty(1, np.uint16)
+    lib().oracle_quant_fp8(_p(x), _p(c), _p(s))
+    return c, s
+
+
+def quant_nvfp4(x: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """256-vector -> (E2M1 codes uint8[256] in 0..15, E4M3 block scales uint16[16])."""
+    x = np.ascontiguousarray(x, np.float32).reshape(256)
+    c = np.empty(256, np.uint8)
+    s = np.empty(16, np.uint16)
+    lib().oracle_quant_nvfp4(_p(x), _p(c), _p(s))
+    return c, s
+
+
+QUANT = {"i8": quant_int8, "q4": quant_q4_0, "e4m3": quant_fp8, "e2m1": quant_nvfp4}
+
+
+def _part(p) -> str:
+    """A part name; True / False stand for "q4" / "i8"."""
+    if isinstance(p, (bool, np.bool_)):
+        return "q4" if p else "i8"
+    return p
+
+
+def n_scales(part) -> int:
+    return N_SCALES[_part(part)]
 
 
 def append_rows(fmt: str, k: np.ndarray, v: np.ndarray):
@@ -146,14 +210,14 @@ def append_rows(fmt: str, k: np.ndarray, v: np.ndarray):
     Returns (kc uint8[n,256], ks uint16[n,nk], vc uint8[n,256], vs uint16[n,nv]);
     int8 codes are returned as their two's-complement bytes.
     """
-    kq4, vq4, _, _ = PARTS[fmt]
+    kp, vp, _, _ = PARTS[fmt]
     k = np.ascontiguousarray(k, np.float32).reshape(-1, 256)
     v = np.ascontiguousarray(v, np.float32).reshape(-1, 256)
     n = k.shape[0]
     kc = np.empty((n, 256), np.uint8)
     vc = np.empty((n, 256), np.uint8)
-    ks = np.empty((n, n_scales(kq4)), np.uint16)
-    vs = np.empty((n, n_scales(vq4)), np.uint16)
+    ks = np.empty((n, n_scales(kp)), np.uint16)
+    vs = np.empty((n, n_scales(vp)), np.uint16)
     rc = lib().oracle_append_rows(FMT[fmt], n, _p(k), _p(v), _p(kc), _p(ks), _p(vc), _p(vs))
     assert rc == 0
     return kc, ks, vc, vs
@@ -166,11 +230,12 @@ def q_prepare(fmt: str, q: np.ndarray) -> np.ndarray:
     return out
 
 
-def dequant_rows(is_q4: bool, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+def dequant_rows(part, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    part = _part(part)
     codes = np.ascontiguousarray(codes).view(np.uint8).reshape(-1, 256)
-    scales = np.ascontiguousarray(scales, np.uint16).reshape(codes.shape[0], n_scales(is_q4))
+    scales = np.ascontiguousarray(scales, np.uint16).reshape(codes.shape[0], n_scales(part))
     out = np.empty((codes.shape[0], 256), np.float64)
-    lib().oracle_dequant_rows(1 if is_q4 else 0, codes.shape[0], _p(codes), _p(scales), _p(out))
+    lib().oracle_dequant_rows(PART_ID[part], codes.shape[0], _p(codes), _p(scales), _p(out))
     return out
 
 

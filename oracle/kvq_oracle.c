@@ -35,6 +35,17 @@
  *    -127, 127), all codes 0 when d rounds to zero.
  *  - Softmax scale 1/sqrt(256) = 1/16.  Q is rotated (q4_0) but never quantised.
  *  - q4_0: K and V rotated; k8v4: V rotated, K not; int8: nothing rotated.
+ *  - fp8 ([Roundup] section 一: 516 bytes per position = 2 x (256 + 2)): each
+ *    256-vector as OCP FP8 E4M3 codes with one fp16 scale d = fp16(max|x| / 448)
+ *    (448 = the largest finite E4M3 value); code = E4M3(x / d), round to
+ *    nearest even, saturating to +-448; all codes +0 when d rounds to zero.
+ *    Not rotated.
+ *  - nvfp4 ([Roundup] section 一: 288 bytes per position = 2 x (128 + 16)):
+ *    blocks of 16 values as E2M1 codes (values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and
+ *    their negatives) with one E4M3 scale per block, s = E4M3(max|x| / 6)
+ *    (round to nearest even, saturating); code = E2M1(x / s), round to nearest
+ *    even, saturating to +-6; all codes +0 when s is zero.  No per-tensor
+ *    scale (it is not in the 288 bytes).  Not rotated.
  */
 #include <math.h>
 #include <stdint.h>
@@ -43,7 +54,19 @@
 
 #define D 256
 
-enum { ORACLE_INT8 = 0, ORACLE_Q4_0 = 1, ORACLE_K8V4 = 2 };
+enum { ORACLE_INT8 = 0, ORACLE_Q4_0 = 1, ORACLE_K8V4 = 2, ORACLE_FP8 = 3, ORACLE_NVFP4 = 4 };
+/* how one half (K or V) of a token-kvhead is stored */
+enum { PART_INT8 = 0, PART_Q4_0 = 1, PART_E4M3 = 2, PART_E2M1 = 3 };
+
+static int part_n_scales(int part)
+{
+    switch (part) {
+    case PART_INT8: return 4;
+    case PART_Q4_0: return 8;
+    case PART_E4M3: return 1;
+    default: return 16;
+    }
+}
 
 /* ---------------------------------------------------------------------------
  * IEEE 754 binary32 -> binary16 / bfloat16, round to nearest, ties to even.
@@ -111,6 +134,83 @@ uint16_t oracle_f32_to_bf16(float f)
     if (rem > 0x8000u || (rem == 0x8000u && (q & 1u)))
         q += 1;                              /* a carry into the exponent is the correct result */
     return (uint16_t)q;
+}
+
+/* ---------------------------------------------------------------------------
+ * OCP 8-bit floating point E4M3 (1 sign, 4 exponent bits with bias 7, 3
+ * fraction bits; no infinities; S.1111.111 is NaN; largest finite 448) and
+ * 4-bit E2M1 (1 sign, 2 exponent bits with bias 1, 1 fraction bit; values
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6), decoded from the field definitions.
+ * ------------------------------------------------------------------------- */
+float oracle_e4m3_to_f32(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);                    /* m/8 * 2^(1-7) */
+    else
+        v = ldexp(8.0 + m, e - 10);                  /* (1 + m/8) * 2^(e-7) */
+    return (float)((b & 0x80) ? -v : v);
+}
+
+float oracle_e2m1_to_f32(uint8_t c)
+{
+    int e = (c >> 1) & 3, m = c & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(2.0 + m, e - 2);   /* (1 + m/2) * 2^(e-1) */
+    return (float)((c & 8) ? -v : v);
+}
+
+/* |x| rounded to nearest, ties to even, on the grid of a small binary format
+ * with `mbits` fraction bits, smallest normal exponent emin and largest finite
+ * value vmax; the result saturates at vmax.  Inside the binade [2^e, 2^(e+1))
+ * (or below 2^emin) the representable values are the multiples of the quantum
+ * 2^(max(e, emin) - mbits), and the binade's first value is an even multiple, so
+ * ties to the even multiple are ties to the even code. */
+static double round_small_format(double a, int mbits, int emin, double vmax)
+{
+    if (a == 0.0)
+        return 0.0;
+    int e;
+    frexp(a, &e);                                    /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                          /* a in [2^e, 2^(e+1)) */
+    if (e < emin)
+        e = emin;
+    double quantum = ldexp(1.0, e - mbits);
+    double r = rint(a / quantum) * quantum;          /* a / quantum is exact (power of two) */
+    return r > vmax ? vmax : r;
+}
+
+/* Field encoding of a value already on the grid (and within range). */
+static uint8_t encode_small_format(double r, int sign, int mbits, int ebits, int bias)
+{
+    int emin = 1 - bias;
+    uint32_t code;
+    if (r < ldexp(1.0, emin)) {                      /* subnormal (or zero) */
+        code = (uint32_t)(r / ldexp(1.0, emin - mbits));
+    } else {
+        int e;
+        frexp(r, &e);
+        e -= 1;
+        uint32_t frac = (uint32_t)((r / ldexp(1.0, e) - 1.0) * (double)(1 << mbits));
+        code = ((uint32_t)(e + bias) << mbits) | frac;
+    }
+    return (uint8_t)((sign ? 1u << (ebits + mbits) : 0u) | code);
+}
+
+uint8_t oracle_f32_to_e4m3(float x)
+{
+    int sign = signbit(x) != 0;
+    double r = round_small_format(fabs((double)x), 3, -6, 448.0);
+    return encode_small_format(r, sign, 3, 4, 7);
+}
+
+uint8_t oracle_f32_to_e2m1(float x)
+{
+    int sign = signbit(x) != 0;
+    double r = round_small_format(fabs((double)x), 1, 0, 6.0);
+    return encode_small_format(r, sign, 1, 2, 1);
 }
 
 /* ---------------------------------------------------------------------------
@@ -205,15 +305,64 @@ void oracle_quant_int8(const float *x, int8_t *codes, uint16_t *scales)
     }
 }
 
+/* fp8: one 256-vector -> 256 E4M3 codes and one fp16 scale.  [Roundup]
+ * section 一 fixes 516 bytes per (layer, KV head) position; the reading is one
+ * fp16 scale per vector for K and for V. */
+void oracle_quant_fp8(const float *x, uint8_t *codes, uint16_t *scale)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < D; ++j)
+        if (fabsf(x[j]) > amax)
+            amax = fabsf(x[j]);
+    float dq = amax / 448.0f;
+    uint16_t dh = oracle_f32_to_f16(dq);
+    *scale = dh;
+    float d = oracle_f16_to_f32(dh);
+    for (int j = 0; j < D; ++j)
+        codes[j] = (d == 0.0f) ? 0 : oracle_f32_to_e4m3(x[j] / d);
+}
+
+/* nvfp4: one 256-vector -> 256 E2M1 codes (0..15, unpacked) and 16 E4M3 block
+ * scales (stored in the low byte of each uint16).  [Roundup] section 一:
+ * 288 bytes per position = 2 x (128 code bytes + 16 scale bytes). */
+void oracle_quant_nvfp4(const float *x, uint8_t *codes, uint16_t *scales)
+{
+    for (int b = 0; b < 16; ++b) {
+        const float *xb = x + 16 * b;
+        float amax = 0.0f;
+        for (int j = 0; j < 16; ++j)
+            if (fabsf(xb[j]) > amax)
+                amax = fabsf(xb[j]);
+        uint8_t sb = oracle_f32_to_e4m3(amax / 6.0f);
+        scales[b] = sb;
+        float sd = oracle_e4m3_to_f32(sb);
+        for (int j = 0; j < 16; ++j)
+            codes[16 * b + j] = (sd == 0.0f) ? 0 : oracle_f32_to_e2m1(xb[j] / sd);
+    }
+}
+
+static void quant_part(int part, const float *x, uint8_t *codes, uint16_t *scales)
+{
+    switch (part) {
+    case PART_INT8: oracle_quant_int8(x, (int8_t *)codes, scales); break;
+    case PART_Q4_0: oracle_quant_q4_0(x, codes, scales); break;
+    case PART_E4M3: oracle_quant_fp8(x, codes, scales); break;
+    default: oracle_quant_nvfp4(x, codes, scales); break;
+    }
+}
+
 /* Layout of one token-kvhead in the oracle's own (unpacked) representation:
- * K codes [256] (uint8 for q4_0, int8 for int8), K scales [8 or 4],
- * V codes [256], V scales [8 or 4].  Returns 0, or -1 for an unknown format. */
-int oracle_format_parts(int fmt, int *k_is_q4, int *v_is_q4, int *k_rot, int *v_rot)
+ * K codes [256] (one byte per value: q4_0 0..15, int8 two's complement, E4M3
+ * bits, E2M1 bits 0..15), K scales [8, 4, 1 or 16] (fp16 bits; E4M3 bits for
+ * nvfp4), then the same for V.  Returns 0, or -1 for an unknown format. */
+int oracle_format_parts(int fmt, int *k_part, int *v_part, int *k_rot, int *v_rot)
 {
     switch (fmt) {
-    case ORACLE_INT8: *k_is_q4 = 0; *v_is_q4 = 0; *k_rot = 0; *v_rot = 0; return 0;
-    case ORACLE_Q4_0: *k_is_q4 = 1; *v_is_q4 = 1; *k_rot = 1; *v_rot = 1; return 0;
-    case ORACLE_K8V4: *k_is_q4 = 0; *v_is_q4 = 1; *k_rot = 0; *v_rot = 1; return 0;
+    case ORACLE_INT8: *k_part = PART_INT8; *v_part = PART_INT8; *k_rot = 0; *v_rot = 0; return 0;
+    case ORACLE_Q4_0: *k_part = PART_Q4_0; *v_part = PART_Q4_0; *k_rot = 1; *v_rot = 1; return 0;
+    case ORACLE_K8V4: *k_part = PART_INT8; *v_part = PART_Q4_0; *k_rot = 0; *v_rot = 1; return 0;
+    case ORACLE_FP8: *k_part = PART_E4M3; *v_part = PART_E4M3; *k_rot = 0; *v_rot = 0; return 0;
+    case ORACLE_NVFP4: *k_part = PART_E2M1; *v_part = PART_E2M1; *k_rot = 0; *v_rot = 0; return 0;
     default: return -1;
     }
 }
@@ -224,14 +373,14 @@ int oracle_format_parts(int fmt, int *k_is_q4, int *v_is_q4, int *k_rot, int *v_
 int oracle_append_token(int fmt, const float *k, const float *v,
                         uint8_t *kc, uint16_t *ks, uint8_t *vc, uint16_t *vs)
 {
-    int kq4, vq4, krot, vrot;
-    if (oracle_format_parts(fmt, &kq4, &vq4, &krot, &vrot))
+    int kpart, vpart, krot, vrot;
+    if (oracle_format_parts(fmt, &kpart, &vpart, &krot, &vrot))
         return -1;
     float tk[D], tv[D];
     if (krot) oracle_fwht256_f32(k, tk); else memcpy(tk, k, sizeof tk);
     if (vrot) oracle_fwht256_f32(v, tv); else memcpy(tv, v, sizeof tv);
-    if (kq4) oracle_quant_q4_0(tk, kc, ks); else oracle_quant_int8(tk, (int8_t *)kc, ks);
-    if (vq4) oracle_quant_q4_0(tv, vc, vs); else oracle_quant_int8(tv, (int8_t *)vc, vs);
+    quant_part(kpart, tk, kc, ks);
+    quant_part(vpart, tv, vc, vs);
     return 0;
 }
 
@@ -239,10 +388,10 @@ int oracle_append_token(int fmt, const float *k, const float *v,
 int oracle_append_rows(int fmt, long n, const float *k, const float *v,
                        uint8_t *kc, uint16_t *ks, uint8_t *vc, uint16_t *vs)
 {
-    int kq4, vq4, krot, vrot;
-    if (oracle_format_parts(fmt, &kq4, &vq4, &krot, &vrot))
+    int kpart, vpart, krot, vrot;
+    if (oracle_format_parts(fmt, &kpart, &vpart, &krot, &vrot))
         return -1;
-    int nks = kq4 ? 8 : 4, nvs = vq4 ? 8 : 4;
+    int nks = part_n_scales(kpart), nvs = part_n_scales(vpart);
     for (long i = 0; i < n; ++i)
         oracle_append_token(fmt, k + D * i, v + D * i, kc + D * i, ks + nks * i, vc + D * i, vs + nvs * i);
     return 0;
@@ -251,8 +400,8 @@ int oracle_append_rows(int fmt, long n, const float *k, const float *v,
 /* Query preparation: the same rotation as K (q4_0 only), never quantised. */
 int oracle_q_prepare(int fmt, const float *q, float *qp, long n_vec)
 {
-    int kq4, vq4, krot, vrot;
-    if (oracle_format_parts(fmt, &kq4, &vq4, &krot, &vrot))
+    int kpart, vpart, krot, vrot;
+    if (oracle_format_parts(fmt, &kpart, &vpart, &krot, &vrot))
         return -1;
     for (long i = 0; i < n_vec; ++i) {
         if (krot) oracle_fwht256_f32(q + D * i, qp + D * i);
@@ -261,24 +410,31 @@ int oracle_q_prepare(int fmt, const float *q, float *qp, long n_vec)
     return 0;
 }
 
-/* Dequantisation to fp64: q4_0 (c - 8) * d, int8 c * d, d the fp16 scale. */
-static void dequant_row(int is_q4, const uint8_t *c, const uint16_t *s, double *out)
+/* Dequantisation to fp64: q4_0 (c - 8) * d, int8 c * d, fp8 E4M3(c) * d
+ * (d the fp16 scale), nvfp4 E2M1(c) * E4M3(s) per block of 16. */
+static void dequant_row(int part, const uint8_t *c, const uint16_t *s, double *out)
 {
-    if (is_q4) {
+    if (part == PART_Q4_0) {
         for (int j = 0; j < D; ++j)
             out[j] = (double)((int)c[j] - 8) * (double)oracle_f16_to_f32(s[j / 32]);
-    } else {
+    } else if (part == PART_INT8) {
         const int8_t *ci = (const int8_t *)c;
         for (int j = 0; j < D; ++j)
             out[j] = (double)ci[j] * (double)oracle_f16_to_f32(s[j / 64]);
+    } else if (part == PART_E4M3) {
+        for (int j = 0; j < D; ++j)
+            out[j] = (double)oracle_e4m3_to_f32(c[j]) * (double)oracle_f16_to_f32(s[0]);
+    } else {
+        for (int j = 0; j < D; ++j)
+            out[j] = (double)oracle_e2m1_to_f32(c[j]) * (double)oracle_e4m3_to_f32((uint8_t)s[j / 16]);
     }
 }
 
-void oracle_dequant_rows(int is_q4, long n, const uint8_t *c, const uint16_t *s, double *out)
+void oracle_dequant_rows(int part, long n, const uint8_t *c, const uint16_t *s, double *out)
 {
-    int ns = is_q4 ? 8 : 4;
+    int ns = part_n_scales(part);
     for (long i = 0; i < n; ++i)
-        dequant_row(is_q4, c + D * i, s + ns * i, out + D * i);
+        dequant_row(part, c + D * i, s + ns * i, out + D * i);
 }
 
 /* Partial attention over tokens [t0, t1) of one KV head for G query heads:
@@ -290,17 +446,17 @@ int oracle_attn_partial(int fmt, const float *qp, int G, long t0, long t1,
                         const uint8_t *vc, const uint16_t *vs,
                         double *m, double *l, double *o)
 {
-    int kq4, vq4, krot, vrot;
-    if (oracle_format_parts(fmt, &kq4, &vq4, &krot, &vrot) || G <= 0 || t1 <= t0)
+    int kpart, vpart, krot, vrot;
+    if (oracle_format_parts(fmt, &kpart, &vpart, &krot, &vrot) || G <= 0 || t1 <= t0)
         return -1;
-    int nks = kq4 ? 8 : 4, nvs = vq4 ? 8 : 4;
+    int nks = part_n_scales(kpart), nvs = part_n_scales(vpart);
     long T = t1 - t0;
     double *s = (double *)malloc(sizeof(double) * (size_t)G * (size_t)T);
     if (!s)
         return -2;
     double row[D];
     for (long t = 0; t < T; ++t) {
-        dequant_row(kq4, kc + D * (t0 + t), ks + nks * (t0 + t), row);
+        dequant_row(kpart, kc + D * (t0 + t), ks + nks * (t0 + t), row);
         for (int h = 0; h < G; ++h) {
             double acc = 0.0;
             for (int j = 0; j < D; ++j)
@@ -325,7 +481,7 @@ int oracle_attn_partial(int fmt, const float *qp, int G, long t0, long t1,
             o[D * h + j] = 0.0;
     }
     for (long t = 0; t < T; ++t) {
-        dequant_row(vq4, vc + D * (t0 + t), vs + nvs * (t0 + t), row);
+        dequant_row(vpart, vc + D * (t0 + t), vs + nvs * (t0 + t), row);
         for (int h = 0; h < G; ++h) {
             double p = s[(size_t)h * T + t];
             for (int j = 0; j < D; ++j)
@@ -353,8 +509,8 @@ void oracle_merge_partials(int G, double *ma, double *la, double *oa,
 /* Final output from a (merged) partial: o / l, then H_n o for rotated V. */
 int oracle_finish(int fmt, int G, const double *l, const double *o, double *out)
 {
-    int kq4, vq4, krot, vrot;
-    if (oracle_format_parts(fmt, &kq4, &vq4, &krot, &vrot))
+    int kpart, vpart, krot, vrot;
+    if (oracle_format_parts(fmt, &kpart, &vpart, &krot, &vrot))
         return -1;
     for (int h = 0; h < G; ++h) {
         double tmp[D];
@@ -395,15 +551,18 @@ double oracle_kv_cache_bytes(int layers, int kv_heads, int head_dim, double byte
     return 2.0 * layers * kv_heads * head_dim * bytes_per_elem * context;
 }
 
-/* Bytes of K and V (codes + fp16 scales) per token per KV head per layer.
+/* Bytes of K and V (codes + scales) per token per KV head per layer.
  * int8: 2 x (256 + 4 x 2) = 528; q4_0: 2 x (128 + 8 x 2) = 288;
- * k8v4: (256 + 4 x 2) + (128 + 8 x 2) = 408. */
+ * k8v4: (256 + 4 x 2) + (128 + 8 x 2) = 408; fp8: 2 x (256 + 2) = 516;
+ * nvfp4: 2 x (128 + 16 x 1) = 288. */
 long oracle_format_bytes_per_token_head(int fmt)
 {
     switch (fmt) {
     case ORACLE_INT8: return 2 * (256 + 4 * 2);
     case ORACLE_Q4_0: return 2 * (128 + 8 * 2);
     case ORACLE_K8V4: return (256 + 4 * 2) + (128 + 8 * 2);
+    case ORACLE_FP8: return 2 * (256 + 1 * 2);
+    case ORACLE_NVFP4: return 2 * (128 + 16 * 1);
     default: return -1;
     }
 }

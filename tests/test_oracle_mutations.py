@@ -36,11 +36,23 @@ MUTATIONS = {
                             "out[j] = (double)ci[j] * (double)oracle_f16_to_f32(s[j / 32 % 4]);"),
     "softmax_scale": ("s[(size_t)h * T + t] = acc / 16.0;", "s[(size_t)h * T + t] = acc / 8.0;"),
     "no_max_subtraction_merge": ("la[h] = la[h] * fa + lb[h] * fb;", "la[h] = la[h] + lb[h] * fb;"),
-    "k8v4_rotates_k": ("case ORACLE_K8V4: *k_is_q4 = 0; *v_is_q4 = 1; *k_rot = 0; *v_rot = 1; return 0;",
-                       "case ORACLE_K8V4: *k_is_q4 = 0; *v_is_q4 = 1; *k_rot = 1; *v_rot = 1; return 0;"),
+    "k8v4_rotates_k": ("case ORACLE_K8V4: *k_part = PART_INT8; *v_part = PART_Q4_0; *k_rot = 0; *v_rot = 1; return 0;",
+                       "case ORACLE_K8V4: *k_part = PART_INT8; *v_part = PART_Q4_0; *k_rot = 1; *v_rot = 1; return 0;"),
     "no_unrotation": ("if (vrot) oracle_fwht256_f64(tmp, out + D * h);", "if (0) oracle_fwht256_f64(tmp, out + D * h);"),
     "q8_bytes": ("case ORACLE_Q4_0: return 2 * (128 + 8 * 2);", "case ORACLE_Q4_0: return 2 * (128 + 4 * 2);"),
+    # fp8 / nvfp4 codecs
+    "e4m3_bias": ("v = ldexp(8.0 + m, e - 10);", "v = ldexp(8.0 + m, e - 9);"),
+    "e4m3_subnormal_step": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "small_format_no_saturation": ("return r > vmax ? vmax : r;", "return r;"),
+    "small_format_ties_away": ("double r = rint(a / quantum) * quantum;", "double r = round(a / quantum) * quantum;"),
+    "e2m1_exponent": ("double v = (e == 0) ? 0.5 * m : ldexp(2.0 + m, e - 2);",
+                      "double v = (e == 0) ? 0.5 * m : ldexp(2.0 + m, e - 1);"),
+    "fp8_divisor": ("float dq = amax / 448.0f;", "float dq = amax / 240.0f;"),
+    "nvfp4_divisor": ("uint8_t sb = oracle_f32_to_e4m3(amax / 6.0f);", "uint8_t sb = oracle_f32_to_e4m3(amax / 4.0f);"),
+    "nvfp4_block_32": ("(double)oracle_e4m3_to_f32((uint8_t)s[j / 16]);", "(double)oracle_e4m3_to_f32((uint8_t)s[j / 32]);"),
+    "fp8_bytes": ("case ORACLE_FP8: return 2 * (256 + 1 * 2);", "case ORACLE_FP8: return 2 * (256 + 2 * 2);"),
 }
+PIN_FILES = ("test_oracle_pins.py", "test_oracle_fp_formats.py")
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
@@ -55,7 +67,7 @@ def test_planted_mistake_is_caught(name):
         subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-o", so, csrc, "-lm"],
                        check=True)
         env = dict(os.environ, KVQ_ORACLE_LIB=so)
-        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] +
+                           [os.path.join(ROOT, "tests", f) for f in PIN_FILES],
                            env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"mutation {name} survived the pins:\n{r.stdout[-2000:]}"

@@ -211,13 +211,13 @@ def test_append_formats_compose_rotation_and_codec():
     rng = np.random.default_rng(6)
     k = rng.standard_normal((3, 256)).astype(np.float32)
     v = rng.standard_normal((3, 256)).astype(np.float32)
-    for fmt, (kq4, vq4, krot, vrot) in oracle.PARTS.items():
+    for fmt, (kp, vp, krot, vrot) in oracle.PARTS.items():
         kc, ks, vc, vs = oracle.append_rows(fmt, k, v)
         for i in range(3):
             kk = oracle.fwht256_f32(k[i])[0] if krot else k[i]
             vv = oracle.fwht256_f32(v[i])[0] if vrot else v[i]
-            ck, sk = (oracle.quant_q4_0 if kq4 else oracle.quant_int8)(kk)
-            cv, sv = (oracle.quant_q4_0 if vq4 else oracle.quant_int8)(vv)
+            ck, sk = oracle.QUANT[kp](kk)
+            cv, sv = oracle.QUANT[vp](vv)
             assert np.array_equal(kc[i], ck.view(np.uint8)) and np.array_equal(ks[i], sk)
             assert np.array_equal(vc[i], cv.view(np.uint8)) and np.array_equal(vs[i], sv)
     # q4_0 rotates Q with the same transform; the other formats leave it alone
@@ -225,6 +225,8 @@ def test_append_formats_compose_rotation_and_codec():
     assert np.array_equal(oracle.q_prepare("q4_0", q), oracle.fwht256_f32(q))
     assert np.array_equal(oracle.q_prepare("int8", q), q)
     assert np.array_equal(oracle.q_prepare("k8v4", q), q)
+    assert np.array_equal(oracle.q_prepare("fp8", q), q)
+    assert np.array_equal(oracle.q_prepare("nvfp4", q), q)
 
 
 # --------------------------------------------------------------------------
@@ -245,7 +247,7 @@ def _sdpa(qp, khat, vhat):
     return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[0, :, 0].numpy()
 
 
-@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
 @pytest.mark.parametrize("T", [1, 7, 300])
 def test_attention_matches_torch_sdpa_fp64(fmt, T):
     rng = np.random.default_rng(10 + T)
@@ -305,7 +307,7 @@ def test_attention_dominant_token():
     assert np.allclose(got[0], oracle.dequant_rows(False, vc[17:18], vs[17:18])[0], rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
 def test_attention_split_invariance_and_permutation(fmt):
     rng = np.random.default_rng(15)
     T = 97
