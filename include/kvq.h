@@ -67,12 +67,19 @@ extern "C" {
 #define KVQ_PAGE_TOKENS 256
 #define KVQ_MAX_GROUP 8          /* query heads per KV head handled by one CTA */
 
-/* KV formats ([Strata] "三种 KV 格式横向对比"):
+/* KV formats ([Strata] "三种 KV 格式横向对比"; [Roundup] section 一 for the
+ * two floating-point formats and their 516 / 288 bytes per position):
  *  KVQ_INT8  K and V int8, one fp16 scale per 64 values, no rotation.
  *  KVQ_Q4_0  K and V rotated by H/16, then q4_0: one fp16 scale per 32 values,
  *            codes 0..15 stored as nibbles ([Guide] "二" q4_0 block).
- *  KVQ_K8V4  K int8 unrotated, V rotated then q4_0. */
-typedef enum { KVQ_INT8 = 0, KVQ_Q4_0 = 1, KVQ_K8V4 = 2 } kvq_format;
+ *  KVQ_K8V4  K int8 unrotated, V rotated then q4_0.
+ *  KVQ_FP8   K and V as FP8 E4M3 codes with one fp16 scale per 256-vector,
+ *            d = fp16(max|x| / 448), code = E4M3(x / d) (round to nearest
+ *            even, saturating); no rotation.
+ *  KVQ_NVFP4 K and V as FP4 E2M1 codes with one E4M3 scale per 16 values,
+ *            s = E4M3(max|x| / 6), code = E2M1(x / s) (round to nearest even,
+ *            saturating); no per-tensor scale; no rotation. */
+typedef enum { KVQ_INT8 = 0, KVQ_Q4_0 = 1, KVQ_K8V4 = 2, KVQ_FP8 = 3, KVQ_NVFP4 = 4 } kvq_format;
 
 typedef struct {
     int32_t n_layers;     /* layers stored in the pool */
@@ -195,7 +202,7 @@ int kvq_decode_plan(const kvq_pool_desc *desc, int n_seq, const int32_t *seq_len
  * a group share one read of each K/V tile.  Writes, per unit, the unnormalised
  * partial output and its running max and sum to the workspace.
  *  q          device fp32 [n_seq][n_q_heads][256]; for q4_0 the output of
- *             q_rotate, for int8 and k8v4 the plain query
+ *             q_rotate, for the other formats the plain query
  *  page_table device int32 [n_seq][max_pages]
  *  plan       device copy of the kvq_decode_plan array; info its host info
  *             (an info whose workspace size differs from the one
@@ -215,6 +222,12 @@ int paged_decode_attn_q4_0(const kvq_pool *pool, int layer, const float *q, cons
 int paged_decode_attn_k8v4(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                            int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                            uint64_t workspace_bytes, int32_t *status, void *stream);
+int paged_decode_attn_fp8(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                          int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                          uint64_t workspace_bytes, int32_t *status, void *stream);
+int paged_decode_attn_nvfp4(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                            int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                            uint64_t workspace_bytes, int32_t *status, void *stream);
 
 /* paged_decode_attn_<fmt>_combined: the same decode with attn_combine fused
  * into it; out_bf16 / out_f32 are written exactly as attn_combine would (merge,
@@ -243,10 +256,18 @@ int paged_decode_attn_k8v4_combined(const kvq_pool *pool, int layer, const float
                                     int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                                     uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
                                     void *stream);
+int paged_decode_attn_fp8_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                   int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                                   uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
+                                   void *stream);
+int paged_decode_attn_nvfp4_combined(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
+                                     int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
+                                     uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status,
+                                     void *stream);
 
 /* paged_decode_step_<fmt>: one whole decode step of one layer in a single
  * launch: kv_append of every sequence's newest token, q_rotate of the raw
- * query (q4_0; int8 and k8v4 take the query as it is) and
+ * query (q4_0; the other formats take the query as it is) and
  * paged_decode_attn_<fmt>_combined over the updated cache.  The results, pool
  * bytes and outputs, are bit-identical to those three calls.
  *  q         device fp32 [n_seq][n_q_heads][256], the raw query
@@ -272,6 +293,14 @@ int paged_decode_step_k8v4(const kvq_pool *pool, int layer, const float *q, cons
                            const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
                            float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
                            int32_t *status, void *stream);
+int paged_decode_step_fp8(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,
+                          const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
+                          float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
+                          int32_t *status, void *stream);
+int paged_decode_step_nvfp4(const kvq_pool *pool, int layer, const float *q, const float *k_new, const float *v_new,
+                            const int32_t *page_table, int max_pages, const int32_t *plan, const kvq_plan_info *info,
+                            float *workspace, uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32,
+                            int32_t *status, void *stream);
 
 /* paged_decode_attn_q4_0_noalloc: paged_decode_attn_q4_0_combined without a
  * workspace argument, for callers that cannot allocate device memory.  Some
@@ -302,7 +331,8 @@ int paged_decode_attn_q4_0_noalloc(const kvq_pool *pool, int layer, const float 
 
 /* The same computation on CUDA cores only (fp32 FMA, no tensor cores).  Kept
  * as the measured control for the tensor-core kernels above; fmt selects the
- * format. */
+ * format (KVQ_INT8, KVQ_Q4_0 or KVQ_K8V4; KVQ_EUNSUPPORTED for KVQ_FP8 and
+ * KVQ_NVFP4, which only the tensor-core path decodes). */
 int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const float *q,
                                const int32_t *page_table, int max_pages, const int32_t *plan,
                                const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,

@@ -162,7 +162,7 @@ class Workload:
     """One synthetic workload: shapes, format and value recipe."""
     name: str
     index: int                  # 1-based position in the workload list
-    fmt: str                    # 'int8' | 'q4_0' | 'k8v4'
+    fmt: str                    # 'int8' | 'q4_0' | 'k8v4' | 'fp8' | 'nvfp4'
     n_layers: int
     n_q_heads: int
     n_kv_heads: int
@@ -293,6 +293,16 @@ WORKLOADS: Dict[str, Workload] = {
                        seq_lens=[8192, 65536, 200000, 262144], page_order="permuted", n_outlier=8,
                        outlier_kind="student_t", q_post=1.0 / 16, q_outliers=False,
                        description="4 ragged sequences, shared pool, random page-to-slot map, k8v4"),
+    # the two floating-point formats the smzdm roundup measures (FP8 516 B and
+    # NVFP4 288 B per position) on the same 27B full-window shape
+    "qwen27b_fp8_262k": _w(name="qwen27b_fp8_262k", index=6, fmt="fp8", n_layers=16, n_q_heads=24, n_kv_heads=4,
+                           seq_lens=[262144], page_order="contiguous", n_outlier=8, outlier_kind="student_t",
+                           q_post=1.0 / 16, q_outliers=False,
+                           description="27B shape at the full 262,144 window, fp8 E4M3 KV, one fp16 scale per vector"),
+    "qwen27b_nvfp4_262k": _w(name="qwen27b_nvfp4_262k", index=7, fmt="nvfp4", n_layers=16, n_q_heads=24,
+                             n_kv_heads=4, seq_lens=[262144], page_order="contiguous", n_outlier=8,
+                             outlier_kind="student_t", q_post=1.0 / 16, q_outliers=False,
+                             description="27B shape at the full 262,144 window, nvfp4 KV (E2M1 + E4M3 per 16)"),
 }
 
 

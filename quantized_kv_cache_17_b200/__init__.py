@@ -7,7 +7,7 @@ missing, importing the binding's functions raises ``KVQError`` at once: there
 is no fallback implementation.
 
 Names follow the C ABI in ``include/kvq.h``: ``q_rotate``, ``kv_append``,
-``paged_decode_attn_{int8,q4_0,k8v4}``, ``attn_combine`` plus the host
+``paged_decode_attn_{int8,q4_0,k8v4,fp8,nvfp4}``, ``attn_combine`` plus the host
 helpers ``pool_bytes``, ``pool_layout`` and ``decode_plan``.
 """
 from __future__ import annotations
@@ -22,8 +22,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
-INT8, Q4_0, K8V4 = 0, 1, 2
-FORMATS = {"int8": INT8, "q4_0": Q4_0, "k8v4": K8V4}
+INT8, Q4_0, K8V4, FP8, NVFP4 = 0, 1, 2, 3, 4
+FORMATS = {"int8": INT8, "q4_0": Q4_0, "k8v4": K8V4, "fp8": FP8, "nvfp4": NVFP4}
 HEAD_DIM = 256
 PAGE_TOKENS = 256
 
@@ -34,9 +34,13 @@ ERRORS = {-1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_EALIGN", -4: "KVQ_E
 EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_append", "kv_append_q_rotate",
            "kvq_decode_plan",
            "paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4",
+           "paged_decode_attn_fp8", "paged_decode_attn_nvfp4",
            "paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined", "paged_decode_attn_k8v4_combined",
+           "paged_decode_attn_fp8_combined", "paged_decode_attn_nvfp4_combined",
            "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine",
-           "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4"]
+           "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4",
+           "paged_decode_step_fp8", "paged_decode_step_nvfp4"]
+_FMT_NAMES = ("int8", "q4_0", "k8v4", "fp8", "nvfp4")
 
 
 class KVQError(RuntimeError):
@@ -84,17 +88,14 @@ def lib():
         L.kv_append_q_rotate.argtypes = [ctypes.POINTER(Pool), I32, P, P, I64, P, P, P, I32, I32, P, P, I64, P, P]
         L.kvq_decode_plan.argtypes = [ctypes.POINTER(PoolDesc), I32, P, I32, I32, P, I32, ctypes.POINTER(PlanInfo)]
         dec = [ctypes.POINTER(Pool), I32, P, P, I32, P, ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P]
-        for n in ("paged_decode_attn_int8", "paged_decode_attn_q4_0", "paged_decode_attn_k8v4"):
-            getattr(L, n).argtypes = dec
-        for n in ("paged_decode_attn_int8_combined", "paged_decode_attn_q4_0_combined",
-                  "paged_decode_attn_k8v4_combined"):
-            getattr(L, n).argtypes = dec[:-2] + [P, P] + dec[-2:]
+        for f in _FMT_NAMES:
+            getattr(L, "paged_decode_attn_" + f).argtypes = dec
+            getattr(L, "paged_decode_attn_" + f + "_combined").argtypes = dec[:-2] + [P, P] + dec[-2:]
         L.paged_decode_attn_q4_0_noalloc.argtypes = dec[:7] + [P, P, P, P]
         L.paged_decode_attn_cudacore.argtypes = [I32] + dec
-        for n in ("paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4"):
-            getattr(L, n).argtypes = [ctypes.POINTER(Pool), I32, P, P, P, P, I32, P, ctypes.POINTER(PlanInfo), P,
-                                      ctypes.c_uint64,
-                                      P, P, P, P]
+        for f in _FMT_NAMES:
+            getattr(L, "paged_decode_step_" + f).argtypes = [ctypes.POINTER(Pool), I32, P, P, P, P, I32, P,
+                                                             ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P, P, P]
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
         for n in EXPORTS[1:]:
             getattr(L, n).restype = ctypes.c_int
@@ -200,7 +201,7 @@ def decode_plan(desc: PoolDesc, seq_lens: Sequence[int], max_pages: int, n_ctas:
     return plan, info
 
 
-_DECODE = {INT8: "paged_decode_attn_int8", Q4_0: "paged_decode_attn_q4_0", K8V4: "paged_decode_attn_k8v4"}
+_DECODE = {FORMATS[f]: "paged_decode_attn_" + f for f in _FMT_NAMES}
 NOALLOC_WS_BYTES = 8 << 20
 
 
@@ -227,7 +228,7 @@ def paged_decode_attn_combined(pool: KVPool, layer: int, q, page_table, plan_dev
                                 _ptr(status), _stream(stream)), name)
 
 
-_STEP = {INT8: "paged_decode_step_int8", Q4_0: "paged_decode_step_q4_0", K8V4: "paged_decode_step_k8v4"}
+_STEP = {FORMATS[f]: "paged_decode_step_" + f for f in _FMT_NAMES}
 
 
 def paged_decode_step(pool: KVPool, layer: int, q, k_new, v_new, page_table, plan_dev, info: PlanInfo, workspace,
@@ -269,6 +270,16 @@ def paged_decode_attn_q4_0(pool, layer, q, page_table, plan_dev, info, workspace
 
 def paged_decode_attn_k8v4(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
     assert pool.fmt == K8V4
+    paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def paged_decode_attn_fp8(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
+    assert pool.fmt == FP8
+    paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def paged_decode_attn_nvfp4(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
+    assert pool.fmt == NVFP4
     paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
 
 

@@ -15,7 +15,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_desc(const kvq_pool_desc *d) {
     if (!d) return KVQ_EINVAL;
     if (d->n_layers <= 0 || d->n_kv_heads <= 0 || d->n_q_heads <= 0 || d->n_pages <= 0) return KVQ_EINVAL;
-    if (d->fmt != KVQ_INT8 && d->fmt != KVQ_Q4_0 && d->fmt != KVQ_K8V4) return KVQ_EINVAL;
+    if (!host_valid_format(d->fmt)) return KVQ_EINVAL;
     if (d->head_dim != KVQ_HEAD_DIM || d->page_tokens != KVQ_PAGE_TOKENS) return KVQ_EUNSUPPORTED;
     if (d->n_q_heads % d->n_kv_heads != 0) return KVQ_EINVAL;
     if (d->n_q_heads / d->n_kv_heads > KVQ_MAX_GROUP) return KVQ_EUNSUPPORTED;
@@ -96,7 +96,7 @@ int decode_common(int fmt, bool tc, const kvq_pool *pool, int layer, const float
     const int rc = check_decode_args(fmt, pool, layer, q, page_table, max_pages, plan, info, workspace_bytes,
                                      out_bf16, out_f32, &geo);
     if (rc) return rc;
-    const int inverse = fmt == KVQ_INT8 ? 0 : 1;
+    const int inverse = host_rotated_v(fmt) ? 1 : 0;
     return cuda_rc(launch_decode(fmt, tc, static_cast<const uint8_t *>(pool->base), geo, layer, q, page_table,
                                  max_pages, plan, *info, workspace, status, inverse, out_bf16, out_f32,
                                  static_cast<cudaStream_t>(stream), k_new, v_new));
@@ -263,10 +263,25 @@ int paged_decode_attn_k8v4(const kvq_pool *pool, int layer, const float *q, cons
                          workspace_bytes, status, stream);
 }
 
+int paged_decode_attn_fp8(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table, int max_pages,
+                          const int32_t *plan, const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,
+                          int32_t *status, void *stream) {
+    return decode_common(KVQ_FP8, true, pool, layer, q, page_table, max_pages, plan, info, workspace,
+                         workspace_bytes, status, stream);
+}
+
+int paged_decode_attn_nvfp4(const kvq_pool *pool, int layer, const float *q, const int32_t *page_table, int max_pages,
+                            const int32_t *plan, const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,
+                            int32_t *status, void *stream) {
+    return decode_common(KVQ_NVFP4, true, pool, layer, q, page_table, max_pages, plan, info, workspace,
+                         workspace_bytes, status, stream);
+}
+
 int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const float *q, const int32_t *page_table,
                                int max_pages, const int32_t *plan, const kvq_plan_info *info, float *workspace,
                                uint64_t workspace_bytes, int32_t *status, void *stream) {
-    if (fmt != KVQ_INT8 && fmt != KVQ_Q4_0 && fmt != KVQ_K8V4) return KVQ_EINVAL;
+    if (!host_valid_format(fmt)) return KVQ_EINVAL;
+    if (fmt == KVQ_FP8 || fmt == KVQ_NVFP4) return KVQ_EUNSUPPORTED;   // the control covers the three 2-part formats
     if (pool) {
         const int G = pool->desc.n_kv_heads > 0 ? pool->desc.n_q_heads / pool->desc.n_kv_heads : 0;
         if (G != 4 && G != 6 && G != 8) return KVQ_EUNSUPPORTED;
@@ -286,6 +301,8 @@ int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const f
 KVQ_COMBINED(paged_decode_attn_int8_combined, KVQ_INT8)
 KVQ_COMBINED(paged_decode_attn_q4_0_combined, KVQ_Q4_0)
 KVQ_COMBINED(paged_decode_attn_k8v4_combined, KVQ_K8V4)
+KVQ_COMBINED(paged_decode_attn_fp8_combined, KVQ_FP8)
+KVQ_COMBINED(paged_decode_attn_nvfp4_combined, KVQ_NVFP4)
 #undef KVQ_COMBINED
 
 #define KVQ_STEP(NAME, FMT)                                                                                     \
@@ -301,6 +318,8 @@ KVQ_COMBINED(paged_decode_attn_k8v4_combined, KVQ_K8V4)
 KVQ_STEP(paged_decode_step_int8, KVQ_INT8)
 KVQ_STEP(paged_decode_step_q4_0, KVQ_Q4_0)
 KVQ_STEP(paged_decode_step_k8v4, KVQ_K8V4)
+KVQ_STEP(paged_decode_step_fp8, KVQ_FP8)
+KVQ_STEP(paged_decode_step_nvfp4, KVQ_NVFP4)
 #undef KVQ_STEP
 
 int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,

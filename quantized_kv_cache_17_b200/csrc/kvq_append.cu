@@ -55,8 +55,11 @@ cudaError_t launch_append_rotate(int fmt, uint8_t *pool, const PoolGeom &geo, in
     const int64_t items = n_rows * geo.n_kv_heads;
     const unsigned ablocks = (unsigned)((items + 3) / 4), rblocks = (unsigned)((n_vec + 3) / 4);
     if (ablocks + rblocks == 0) return cudaSuccess;
-    auto kern = fmt == KVQ_INT8 ? append_rotate_kernel<KVQ_INT8>
-                                : (fmt == KVQ_Q4_0 ? append_rotate_kernel<KVQ_Q4_0> : append_rotate_kernel<KVQ_K8V4>);
+    auto kern = fmt == KVQ_INT8    ? append_rotate_kernel<KVQ_INT8>
+                : fmt == KVQ_Q4_0  ? append_rotate_kernel<KVQ_Q4_0>
+                : fmt == KVQ_K8V4  ? append_rotate_kernel<KVQ_K8V4>
+                : fmt == KVQ_FP8   ? append_rotate_kernel<KVQ_FP8>
+                                   : append_rotate_kernel<KVQ_NVFP4>;
     return launch_ex(kern, dim3(ablocks + rblocks), dim3(128), 0, s, false, pool, geo, layer, k, v, n_rows, row_seq,
                      row_pos, page_table, max_pages, n_seq, status, ablocks, q, q_rot, n_vec);
 }
@@ -67,8 +70,11 @@ cudaError_t launch_append(int fmt, uint8_t *pool, const PoolGeom &geo, int layer
     if (n_rows == 0) return cudaSuccess;
     const int64_t items = n_rows * geo.n_kv_heads;
     const unsigned blocks = (unsigned)((items + 3) / 4);
-    auto kern = fmt == KVQ_INT8 ? append_kernel<KVQ_INT8> : (fmt == KVQ_Q4_0 ? append_kernel<KVQ_Q4_0>
-                                                                                : append_kernel<KVQ_K8V4>);
+    auto kern = fmt == KVQ_INT8    ? append_kernel<KVQ_INT8>
+                : fmt == KVQ_Q4_0  ? append_kernel<KVQ_Q4_0>
+                : fmt == KVQ_K8V4  ? append_kernel<KVQ_K8V4>
+                : fmt == KVQ_FP8   ? append_kernel<KVQ_FP8>
+                                   : append_kernel<KVQ_NVFP4>;
     return launch_ex(kern, dim3(blocks), dim3(128), 0, s, false, pool, geo, layer, k, v, n_rows, row_seq, row_pos,
                      page_table, max_pages, n_seq, status);
 }

@@ -1,6 +1,7 @@
 // Device code of q_rotate and kv_append, shared by the launches that run them
 // on their own and by the decode-step kernel that runs them inside the decode:
-// the 256-point Walsh-Hadamard rotation and the q4_0 / int8 block quantisers,
+// the 256-point Walsh-Hadamard rotation and the q4_0 / int8 / fp8 / nvfp4 block
+// quantisers ([Roundup] section 一 for the last two),
 // written into the fragment-ordered pool layout.
 //
 // [Strata] "4-bit KV 缓存：先旋转，再压到 4-bit": K, V (and the query) are rotated
@@ -119,6 +120,37 @@ __device__ __forceinline__ void quant_i8_lane(const float (&x)[8], int (&c)[8], 
     }
 }
 
+// ---- fp8: one E4M3 code per value, one fp16 scale per 256-vector ------------
+// d = fp16(max|x| / 448); code = E4M3(x / d) (round to nearest even,
+// saturating); all codes +0 when d rounds to zero.
+__device__ __forceinline__ void quant_f8_lane(const float (&x)[8], int (&c)[8], __half &d16) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    d16 = __float2half_rn(__fdiv_rn(amax, 448.0f));
+    const float df = __half2float(d16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = df != 0.0f ? (int)f32_to_e4m3(__fdiv_rn(x[i], df)) : 0;
+}
+
+// ---- nvfp4: blocks of 16 = 2 lanes, E2M1 codes, one E4M3 scale per block ------
+// s = E4M3(max|x| / 6); code = E2M1(x / s) (round to nearest even,
+// saturating); all codes +0 when s is zero.  The scale byte travels in d16's
+// bits.
+__device__ __forceinline__ void quant_f4_lane(const float (&x)[8], int (&c)[8], __half &d16) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const uint32_t sb = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+    d16 = __ushort_as_half((unsigned short)sb);
+    const float sd = __half2float(__ushort_as_half((unsigned short)(e4m3x2_to_h2(sb) & 0xFFFFu)));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = sd != 0.0f ? (int)f32_to_e2m1(__fdiv_rn(x[i], sd)) : 0;
+}
+
 // ---- stores into the fragment-ordered tile ---------------------------------
 // K side, Q4: lane (block b = lane>>2, jl = lane&3) holds dims 32b + 8jl + e.
 // Dim 32b + 8(n&3) + (n>>2) + 2j lives in word W(r,b,j) nibble n, so element
@@ -192,6 +224,24 @@ __device__ __forceinline__ void store_i8_vside(uint8_t *tile, int r, int lane, c
     for (int g = 0; g < 8; ++g) base[g * 64] = (uint8_t)(c[g] & 0xFF);
 }
 
+// K side, F4: word W(r,b,j) (where Q4 puts it) byte q holds dims 32b + 8q + 2j
+// (low nibble) and + 1 (high nibble).  Lane (b = lane>>2, jl = lane&3) holds
+// dims 32b + 8jl + e: byte q = jl of word j = e>>1, nibble e&1.
+__device__ __forceinline__ void store_f4_kside(uint8_t *tile, int r, int lane, const int (&c)[8]) {
+    const int b = lane >> 2, jl = lane & 3;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = ((uint32_t)c[2 * j] | ((uint32_t)c[2 * j + 1] << 4)) << (8 * jl);
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] |= __shfl_xor_sync(0xffffffffu, w[j], m);
+    uint32_t mine = w[0];
+#pragma unroll
+    for (int j = 1; j < 4; ++j) if (jl == j) mine = w[j];
+    *reinterpret_cast<uint32_t *>(tile + (b >> 2) * 512 + (r * 4 + jl) * 16 + (b & 3) * 4) = mine;
+}
+
 __device__ __forceinline__ void store_scale_q4(uint8_t *sc, int r, int lane, __half d) {
     if ((lane & 3) == 0)
         *reinterpret_cast<__half *>(sc + (r >> 1) * 32 + (lane >> 2) * 4 + (r & 1) * 2) = d;
@@ -200,13 +250,28 @@ __device__ __forceinline__ void store_scale_i8(uint8_t *sc, int r, int lane, __h
     if ((lane & 7) == 0)
         *reinterpret_cast<__half *>(sc + (r >> 1) * 16 + (lane >> 3) * 4 + (r & 1) * 2) = d;
 }
+__device__ __forceinline__ void store_scale_f8(uint8_t *sc, int r, int lane, __half d) {
+    if (lane == 0) *reinterpret_cast<__half *>(sc + 2 * r) = d;
+}
+// the E4M3 byte of block lane/2 (both lanes of the block hold it)
+__device__ __forceinline__ void store_scale_f4(uint8_t *sc, int r, int lane, __half d) {
+    if ((lane & 1) == 0) sc[(r >> 1) * 32 + (lane >> 1) * 2 + (r & 1)] = (uint8_t)__half_as_ushort(d);
+}
 
-// A token's codes and fp16 block scales as one lane of the encoding warp holds
-// them (lane l: elements 8l .. 8l+7 of the rotated or plain K and V rows).
+// A token's codes and block scales as one lane of the encoding warp holds them
+// (lane l: elements 8l .. 8l+7 of the rotated or plain K and V rows); an E4M3
+// scale rides in the low byte of the __half's bits.
 struct TokenCodes {
     int k[8], v[8];
     __half dk, dv;
 };
+
+template <int P> __device__ __forceinline__ void quant_part(const float (&x)[8], int lane, int (&c)[8], __half &d) {
+    if constexpr (P == PART_Q4) quant_q4_lane(x, lane, c, d);
+    else if constexpr (P == PART_I8) quant_i8_lane(x, c, d);
+    else if constexpr (P == PART_F8) quant_f8_lane(x, c, d);
+    else quant_f4_lane(x, c, d);
+}
 
 // One warp quantises one token of one KV head: xk / xv = its 256 K and V values
 // (lane l holds 8l .. 8l+7), rotated first where the format stores them rotated.
@@ -214,30 +279,40 @@ template <int FMT>
 __device__ __forceinline__ void quant_token(float (&xk)[8], float (&xv)[8], int lane, TokenCodes &t) {
     using L = TileLayout<FMT>;
     if (Fmt<FMT>::KROT) fwht256_lane(xk, lane);
-    if (L::KP == PART_Q4) quant_q4_lane(xk, lane, t.k, t.dk);
-    else quant_i8_lane(xk, t.k, t.dk);
+    quant_part<L::KP>(xk, lane, t.k, t.dk);
     if (Fmt<FMT>::VROT) fwht256_lane(xv, lane);
-    if (L::VP == PART_Q4) quant_q4_lane(xv, lane, t.v, t.dv);
-    else quant_i8_lane(xv, t.v, t.dv);
+    quant_part<L::VP>(xv, lane, t.v, t.dv);
 }
 
 // The warp writes the token as row r of the tile at `tile`.
 template <int FMT>
 __device__ __forceinline__ void store_token(const TokenCodes &t, int lane, int r, uint8_t *tile) {
     using L = TileLayout<FMT>;
-    if (L::KP == PART_Q4) {
+    if constexpr (L::KP == PART_Q4) {
         store_q4_kside(tile + L::KC, r, lane, t.k);
         store_scale_q4(tile + L::KS, r, lane, t.dk);
-    } else {
+    } else if constexpr (L::KP == PART_I8) {
         store_i8_kside(tile + L::KC, r, lane, t.k);
         store_scale_i8(tile + L::KS, r, lane, t.dk);
+    } else if constexpr (L::KP == PART_F8) {
+        store_i8_kside(tile + L::KC, r, lane, t.k);
+        store_scale_f8(tile + L::KS, r, lane, t.dk);
+    } else {
+        store_f4_kside(tile + L::KC, r, lane, t.k);
+        store_scale_f4(tile + L::KS, r, lane, t.dk);
     }
-    if (L::VP == PART_Q4) {
+    if constexpr (L::VP == PART_Q4) {
         store_q4_vside(tile + L::VC, r, lane, t.v);
         store_scale_q4(tile + L::VS, r, lane, t.dv);
-    } else {
+    } else if constexpr (L::VP == PART_I8) {
         store_i8_vside(tile + L::VC, r, lane, t.v);
         store_scale_i8(tile + L::VS, r, lane, t.dv);
+    } else if constexpr (L::VP == PART_F8) {
+        store_i8_vside(tile + L::VC, r, lane, t.v);
+        store_scale_f8(tile + L::VS, r, lane, t.dv);
+    } else {
+        store_q4_vside(tile + L::VC, r, lane, t.v);
+        store_scale_f4(tile + L::VS, r, lane, t.dv);
     }
 }
 

@@ -154,15 +154,16 @@ template <int FMT> struct TcCfg {
     static_assert(2 * NQK * REG_COMPUTE + 4 * REG_PROD <= NTHREADS / 32 * REG_LAUNCH,
                   "register split exceeds the launch's registers");
     static_assert(SCALE_WARP + N_SCALE == NTHREADS / 32, "producer warpgroup: copy warp + scale warps");
-    static constexpr int TPI = FMT == KVQ_INT8 ? 2 : 4;         // tiles per work item (measured best)
+    // tiles per work item (measured best for int8 and q4_0; the 8-bit fp8 tiles follow int8)
+    static constexpr int TPI = (FMT == KVQ_INT8 || FMT == KVQ_FP8) ? 2 : 4;
     static constexpr int ITEMS_PER_STAGE = 8 / TPI;
     static constexpr int STAGE_BYTES = 8 * L::BYTES;
-    static constexpr int NS = FMT == KVQ_Q4_0 ? 8 : (FMT == KVQ_INT8 ? 5 : 6);
+    static constexpr int NS = (FMT == KVQ_Q4_0 || FMT == KVQ_NVFP4) ? 8 : ((FMT == KVQ_INT8 || FMT == KVQ_FP8) ? 5 : 6);
     static constexpr int DP = 2;                                // slots of each QK -> PV ring
     // fp32 K scales of a stage: per tile, token pair t at float t*KSTRIDE (block
     // or group j of tokens 2t, 2t+1 at 2j, 2j+1); the stride pads rows so the
     // four pairs fall into different banks
-    static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : 12;
+    static constexpr int KSTRIDE = L::KP == PART_Q4 ? 20 : (L::KP == PART_I8 ? 12 : (L::KP == PART_F8 ? 2 : 36));
     static constexpr int SF_TILE = 4 * KSTRIDE;                 // floats
     static constexpr int SF_STAGE_BYTES = 8 * SF_TILE * 4;
     static constexpr int PA = 32 * 2 * TPI;                     // alpha[8] in a slot, after p of 32 lanes x 2 TPI
@@ -204,16 +205,43 @@ template <int FMT> struct TcCfg {
 // softmax.  The fp32 K scales are therefore stored multiplied by 2^(24 - KBS).
 template <int FMT> struct QkCodes {
     static constexpr bool Q4 = TileLayout<FMT>::KP == PART_Q4;
+    // fp8 / fp4 keys convert to exact fp16 values: no offset, no 2^-24 units
+    static constexpr bool FP = TileLayout<FMT>::KP == PART_F8 || TileLayout<FMT>::KP == PART_F4;
     static constexpr float OFF = Q4 ? 8.f : 128.f;
-    static constexpr int KBS = Q4 ? 6 : 11;
-    static constexpr float KSF = Q4 ? 262144.f : 8192.f;     // 2^(24 - KBS)
+    static constexpr int KBS = FP ? 0 : (Q4 ? 6 : 11);
+    static constexpr float KSF = FP ? 1.f : (Q4 ? 262144.f : 8192.f);     // 2^(24 - KBS)
 };
 
-// Scale warp: convert the fp16 K scales of one stage (8 tiles) to fp32 rows
-// (times 2^(24 - KBS)).
+// Scale warp: convert the K scales of one stage (8 tiles) to fp32 rows (times
+// 2^(24 - KBS) for the 4/8-bit integer codes).  fp8: one fp16 per token, row
+// of pair t = (d[2t], d[2t+1]); nvfp4: 16 E4M3 per token, row of pair t =
+// (d[2t][b], d[2t+1][b]) for b = 0..15.
 template <int FMT>
 __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float *sf, int lane) {
     using L = TileLayout<FMT>;
+    if constexpr (L::KP == PART_F8) {
+        const int tile = lane >> 2, pair = lane & 3;
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(stage + tile * L::BYTES + L::KS + pair * 4);
+        const float2 d = __half22float2(u32_as_h2(w));
+        *reinterpret_cast<float2 *>(sf + tile * TcCfg<FMT>::SF_TILE + pair * TcCfg<FMT>::KSTRIDE) = d;
+        return;
+    } else if constexpr (L::KP == PART_F4) {
+        constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
+#pragma unroll
+        for (int c = lane; c < 8 * 8; c += 32) {            // 8 chunks of 16 bytes per tile
+            const int tile = c >> 3, pair = (c >> 1) & 3, half = c & 1;
+            const uint4 h = lds128(stage + tile * L::BYTES + L::KS + pair * 32 + half * 16);
+            float *dst = sf + tile * 4 * KSTRIDE + pair * KSTRIDE + half * 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t w = u4_at(h, i);
+                const float2 a = __half22float2(u32_as_h2(e4m3x2_to_h2(w)));
+                const float2 b = __half22float2(u32_as_h2(e4m3x2_to_h2(w >> 16)));
+                *reinterpret_cast<float4 *>(dst + 4 * i) = make_float4(a.x, a.y, b.x, b.y);
+            }
+        }
+        return;
+    }
     constexpr int KSB = part_scale_bytes(L::KP);        // fp16 bytes per tile: 4 token pairs
     constexpr int PAIR_B = KSB / 4;                     // 32 (q4) or 16 (i8) bytes per pair
     constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
@@ -250,23 +278,39 @@ __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float
 __device__ __forceinline__ int pv_sigma(int e) { return min(15, 29 - (e > 1 ? e : 1)); }
 
 // The largest |V scale| of the TPI tiles at tp, as fp16 bits (warp-uniform).
-// fp16 magnitudes order as integers.  Tokens past the sequence end count too
-// (their bytes are stale or zero): that can only lower sigma, never overflow.
+// fp16 (and E4M3) magnitudes order as integers.  Tokens past the sequence end
+// count too (their bytes are stale or zero): that can only lower sigma, never
+// overflow.
 template <int FMT> __device__ __forceinline__ uint32_t item_v_scale_max(const uint8_t *tp, int lane) {
     using L = TileLayout<FMT>;
-    constexpr int VSB = part_scale_bytes(L::VP);              // bytes per tile
-    constexpr int PER_LANE = TcCfg<FMT>::TPI * VSB / 32;      // 16 (q4) or 4 (int8) bytes
-    constexpr int LPT = VSB / PER_LANE;                       // lanes per tile
-    const uint8_t *src = tp + (lane / LPT) * L::BYTES + L::VS + (lane % LPT) * PER_LANE;
-    uint32_t m;
-    if constexpr (PER_LANE == 16) {
-        const uint4 h = lds128(src);
-        m = __vmaxu2(__vmaxu2(h.x & 0x7FFF7FFFu, h.y & 0x7FFF7FFFu), __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));
+    if constexpr (L::VP == PART_F8) {                         // one fp16 per token: TPI x 8 of them
+        const uint32_t m = lane < 8 * TcCfg<FMT>::TPI
+                               ? *reinterpret_cast<const uint16_t *>(tp + (lane >> 3) * L::BYTES + L::VS + (lane & 7) * 2) &
+                                     0x7FFFu
+                               : 0u;
+        return __reduce_max_sync(0xffffffffu, m);
+    } else if constexpr (L::VP == PART_F4) {                  // E4M3 bytes, 16 per lane
+        static_assert(TcCfg<FMT>::TPI == 4, "nvfp4: four tiles per item");
+        const uint4 h = lds128(tp + (lane >> 3) * L::BYTES + L::VS + (lane & 7) * 16);
+        uint32_t m = __vmaxu4(__vmaxu4(h.x & 0x7F7F7F7Fu, h.y & 0x7F7F7F7Fu), __vmaxu4(h.z & 0x7F7F7F7Fu, h.w & 0x7F7F7F7Fu));
+        m = max(max(m & 0xFFu, (m >> 8) & 0xFFu), max((m >> 16) & 0xFFu, m >> 24));
+        m = __reduce_max_sync(0xffffffffu, m);
+        return e4m3x2_to_h2(m) & 0xFFFFu;                      // its fp16 bits (exact)
     } else {
-        static_assert(PER_LANE == 4, "V scale bytes per lane");
-        m = *reinterpret_cast<const uint32_t *>(src) & 0x7FFF7FFFu;
+        constexpr int VSB = part_scale_bytes(L::VP);          // bytes per tile
+        constexpr int PER_LANE = TcCfg<FMT>::TPI * VSB / 32;  // 16 (q4) or 4 (int8) bytes
+        constexpr int LPT = VSB / PER_LANE;                   // lanes per tile
+        const uint8_t *src = tp + (lane / LPT) * L::BYTES + L::VS + (lane % LPT) * PER_LANE;
+        uint32_t m;
+        if constexpr (PER_LANE == 16) {
+            const uint4 h = lds128(src);
+            m = __vmaxu2(__vmaxu2(h.x & 0x7FFF7FFFu, h.y & 0x7FFF7FFFu), __vmaxu2(h.z & 0x7FFF7FFFu, h.w & 0x7FFF7FFFu));
+        } else {
+            static_assert(PER_LANE == 4, "V scale bytes per lane");
+            m = *reinterpret_cast<const uint32_t *>(src) & 0x7FFF7FFFu;
+        }
+        return __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
     }
-    return __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
 }
 
 template <int FMT> struct QkWarp {
@@ -335,7 +379,7 @@ template <int FMT> struct QkWarp {
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int b = 0; b < 8; b += 2)
-            if (b == 2 * t && (K::Q4 || b < 4)) {
+            if (b == 2 * t && !K::FP && (K::Q4 || b < 4)) {
                 a0 = CA * S[b];
                 a1 = CA * S[b + 1];
             }
@@ -366,6 +410,64 @@ template <int FMT> struct QkWarp {
         const uint8_t *tB = tA + L::BYTES;
         const float *fB = fA + C::SF_TILE;
         const int t = lane & 3;
+        if constexpr (L::KP == PART_F8) {
+            // E4M3 keys: the 16 k-steps accumulate in two chains per tile; the
+            // token's one scale multiplies the sum
+            float a[2][4], c[2][4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 kA = lds128(tA + L::KC + q * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + q * 512 + lane * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t wA = u4_at(kA, j), wB = u4_at(kB, j);
+                    const uint4 qj = qa(4 * q + j, lane);
+                    float(&ra)[4] = a[q & 1];
+                    float(&rc)[4] = c[q & 1];
+                    if (q < 2 && j == 0) {
+                        mma_z(ra, qj, e4m3x2_to_h2(wA), e4m3x2_to_h2(wA >> 16));
+                        mma_z(rc, qj, e4m3x2_to_h2(wB), e4m3x2_to_h2(wB >> 16));
+                    } else {
+                        mma_acc(ra, qj, e4m3x2_to_h2(wA), e4m3x2_to_h2(wA >> 16));
+                        mma_acc(rc, qj, e4m3x2_to_h2(wB), e4m3x2_to_h2(wB >> 16));
+                    }
+                }
+            }
+            const float2 dA = *reinterpret_cast<const float2 *>(fA + t * C::KSTRIDE);
+            const float2 dB = *reinterpret_cast<const float2 *>(fB + t * C::KSTRIDE);
+            s[0] = ((a[0][0] + a[0][2]) + (a[1][0] + a[1][2])) * dA.x;
+            s[1] = ((a[0][1] + a[0][3]) + (a[1][1] + a[1][3])) * dA.y;
+            s[2] = ((c[0][0] + c[0][2]) + (c[1][0] + c[1][2])) * dB.x;
+            s[3] = ((c[0][1] + c[0][3]) + (c[1][1] + c[1][3])) * dB.y;
+            return;
+        } else if constexpr (L::KP == PART_F4) {
+            // E2M1 keys: one k-step per 16-value block, each with its own scale
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[i] = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 kA = lds128(tA + L::KC + hf * 512 + lane * 16);
+                const uint4 kB = lds128(tB + L::KC + hf * 512 + lane * 16);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int b = 4 * hf + bb;              // 32 dims: k-steps 2b, 2b + 1
+                    const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
+                    float a0[4], a1[4], c0[4], c1[4];
+                    const uint4 q0 = qa(2 * b, lane), q1 = qa(2 * b + 1, lane);
+                    mma_z(a0, q0, e2m1x2_to_h2(wA), e2m1x2_to_h2(wA >> 8));
+                    mma_z(c0, q0, e2m1x2_to_h2(wB), e2m1x2_to_h2(wB >> 8));
+                    mma_z(a1, q1, e2m1x2_to_h2(wA >> 16), e2m1x2_to_h2(wA >> 24));
+                    mma_z(c1, q1, e2m1x2_to_h2(wB >> 16), e2m1x2_to_h2(wB >> 24));
+                    const float4 dA = *reinterpret_cast<const float4 *>(fA + t * C::KSTRIDE + 4 * b);
+                    const float4 dB = *reinterpret_cast<const float4 *>(fB + t * C::KSTRIDE + 4 * b);
+                    s[0] = fmaf(a1[0] + a1[2], dA.z, fmaf(a0[0] + a0[2], dA.x, s[0]));
+                    s[1] = fmaf(a1[1] + a1[3], dA.w, fmaf(a0[1] + a0[3], dA.y, s[1]));
+                    s[2] = fmaf(c1[0] + c1[2], dB.z, fmaf(c0[0] + c0[2], dB.x, s[2]));
+                    s[3] = fmaf(c1[1] + c1[3], dB.w, fmaf(c0[1] + c0[3], dB.y, s[3]));
+                }
+            }
+            return;
+        }
         {
             float ca[4], cb[4];
             mma_k8(ca, qb_hi, qb_lo, kscale_frag(tA, lane));
@@ -542,6 +644,49 @@ template <int FMT> struct PvWarp {
         }
     }
 
+    // E4M3 values: the token's one scale gives one P' pair per tile for every
+    // m-tile; bytes (2t, 2t+1) of a word are one token pair at one dim.
+    __device__ __forceinline__ void pv_f8(int q, const uint4 &wvA, const uint4 &wvB, uint32_t hA, uint32_t lA,
+                                          uint32_t hB, uint32_t lB) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t xa = u4_at(wvA, j), xb = u4_at(wvB, j);
+            const uint4 m = make_uint4(e4m3x2_to_h2(xa), e4m3x2_to_h2(xa >> 16), e4m3x2_to_h2(xb), e4m3x2_to_h2(xb >> 16));
+            mma_acc(o[4 * q + j], m, hA, hB);
+            mma_acc(o[4 * q + j], m, lA, lB);
+        }
+    }
+    // E2M1 values in the q4_0 word order (token 2t in nibbles 0-3, token 2t+1
+    // in nibbles 4-7, dims g, g+8, g+16, g+24): pair the nibbles of the two
+    // tokens per dim into bytes, one cvt.e2m1x2 each.  dv0 / dv1: E4M3 scale
+    // pairs (tokens 2t, 2t+1) of the two 16-dim blocks of 32-dim block b.
+    __device__ __forceinline__ static void f4_pairs(uint32_t w, uint32_t &d0, uint32_t &d8, uint32_t &d16,
+                                                    uint32_t &d24) {
+        const uint32_t a = w & 0x0F0F0F0Fu, b = (w >> 4) & 0x0F0F0F0Fu;
+        const uint32_t u = a | (a >> 12), v = b | (b >> 12);   // bytes: (dim g, dim g+16) and (g+8, g+24)
+        d0 = e2m1x2_to_h2(u);
+        d16 = e2m1x2_to_h2(u >> 8);
+        d8 = e2m1x2_to_h2(v);
+        d24 = e2m1x2_to_h2(v >> 8);
+    }
+    __device__ __forceinline__ void pv_f4(int b, uint32_t wA, uint32_t wB, uint32_t eA, uint32_t eB, uint32_t mA,
+                                          uint32_t mB, uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
+        uint32_t a0, a8, a16, a24, b0, b8, b16, b24;
+        f4_pairs(wA, a0, a8, a16, a24);
+        f4_pairs(wB, b0, b8, b16, b24);
+        uint32_t hA, lA, hB, lB;
+        pscale(e4m3x2_to_h2(eA) & mA, phA, plA, hA, lA);             // block 2b
+        pscale(e4m3x2_to_h2(eB) & mB, phB, plB, hB, lB);
+        const uint4 m0 = make_uint4(a0, a8, b0, b8);
+        mma_acc(o[2 * b], m0, hA, hB);
+        mma_acc(o[2 * b], m0, lA, lB);
+        pscale(e4m3x2_to_h2(eA >> 16) & mA, phA, plA, hA, lA);       // block 2b + 1
+        pscale(e4m3x2_to_h2(eB >> 16) & mB, phB, plB, hB, lB);
+        const uint4 m1 = make_uint4(a16, a24, b16, b24);
+        mma_acc(o[2 * b + 1], m1, hA, hB);
+        mma_acc(o[2 * b + 1], m1, lA, lB);
+    }
+
     // Tiles A, B (consecutive) with p of their tokens 2t, 2t+1.
     template <bool MASK>
     __device__ __forceinline__ void two_tiles(const uint8_t *tA, int vA, int vB, int t, int lane, float pA0, float pA1,
@@ -564,6 +709,29 @@ template <int FMT> struct PvWarp {
                 for (int bb = 0; bb < 4; ++bb)
                     pv_q4(4 * hf + bb, u4_at(wvA, bb), u4_at(wvB, bb), u4_at(eA, bb) & mA, u4_at(eB, bb) & mB, phA,
                           plA, phB, plB);
+            }
+        } else if constexpr (L::VP == PART_F4) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint4 wvA = lds128(tA + L::VC + hf * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + hf * 512 + lane * 16);
+                // E4M3 pairs (dV[2t][blk], dV[2t+1][blk]) for the 16-dim blocks 8 hf .. 8 hf + 7
+                const uint4 eA = lds128(tA + L::VS + t * 32 + hf * 16);
+                const uint4 eB = lds128(tB + L::VS + t * 32 + hf * 16);
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    pv_f4(4 * hf + bb, u4_at(wvA, bb), u4_at(wvB, bb), u4_at(eA, bb), u4_at(eB, bb), mA, mB, phA, plA,
+                          phB, plB);
+            }
+        } else if constexpr (L::VP == PART_F8) {
+            uint32_t hA, lA, hB, lB;
+            pscale(*reinterpret_cast<const uint32_t *>(tA + L::VS + t * 4) & mA, phA, plA, hA, lA);
+            pscale(*reinterpret_cast<const uint32_t *>(tB + L::VS + t * 4) & mB, phB, plB, hB, lB);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 wvA = lds128(tA + L::VC + q * 512 + lane * 16);
+                const uint4 wvB = lds128(tB + L::VC + q * 512 + lane * 16);
+                pv_f8(q, wvA, wvB, hA, lA, hB, lB);
             }
         } else {
             const uint4 eA = lds128(tA + L::VS + t * 16);                 // (dV[2t][q], dV[2t+1][q]), q = 0..3
@@ -1702,11 +1870,16 @@ cudaError_t launch_fmt(bool tc, const DecodeArgs &a, int n_units, cudaStream_t s
         return launch_decode_kernel<decode_tc_kernel<FMT, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s,
                                                                   C::REG_LAUNCH);
     }
-    using C = AluCfg<FMT>;
-    switch (a.G) {
-    case 4: return launch_decode_kernel<decode_alu_kernel<FMT, 4, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
-    case 6: return launch_decode_kernel<decode_alu_kernel<FMT, 6, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
-    default: return launch_decode_kernel<decode_alu_kernel<FMT, 8, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+    if constexpr (FMT == KVQ_FP8 || FMT == KVQ_NVFP4) {
+        return cudaErrorNotSupported;          // the CUDA-core control covers the integer-code formats only
+    } else {
+        using C = AluCfg<FMT>;
+        switch (a.G) {
+        case 4: return launch_decode_kernel<decode_alu_kernel<FMT, 4, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+        case 6: return launch_decode_kernel<decode_alu_kernel<FMT, 6, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+        default:
+            return launch_decode_kernel<decode_alu_kernel<FMT, 8, FUSED>>(C::TOTAL, C::NTHREADS, a, n_units, FUSED, s);
+        }
     }
 }
 
@@ -1715,7 +1888,9 @@ cudaError_t launch_fused(int fmt, bool tc, const DecodeArgs &a, int n_units, cud
     switch (fmt) {
     case KVQ_INT8: return launch_fmt<KVQ_INT8, FUSED>(tc, a, n_units, s);
     case KVQ_Q4_0: return launch_fmt<KVQ_Q4_0, FUSED>(tc, a, n_units, s);
-    default: return launch_fmt<KVQ_K8V4, FUSED>(tc, a, n_units, s);
+    case KVQ_K8V4: return launch_fmt<KVQ_K8V4, FUSED>(tc, a, n_units, s);
+    case KVQ_FP8: return launch_fmt<KVQ_FP8, FUSED>(tc, a, n_units, s);
+    default: return launch_fmt<KVQ_NVFP4, FUSED>(tc, a, n_units, s);
     }
 }
 

@@ -26,12 +26,15 @@ constexpr int WS_TAIL = 16;       // m[8], l[8] after o[G][256] in one workspace
 // Pool layout.
 //
 // pool = [layer][slot][kv_head] page blocks; page block = 32 tiles of 8 tokens;
-// tile = [K codes | K scales | V codes | V scales].  Two kinds of part:
+// tile = [K codes | K scales | V codes | V scales].  Four kinds of part:
 //
-//   Q4 part (q4_0): codes 1024 B (8 tok x 256 x 4 bit), scales 128 B (8 tok x 8 fp16)
-//   I8 part (int8): codes 2048 B (8 tok x 256 x 8 bit), scales  64 B (8 tok x 4 fp16)
+//   Q4 part (q4_0):  codes 1024 B (8 tok x 256 x 4 bit), scales 128 B (8 tok x 8 fp16)
+//   I8 part (int8):  codes 2048 B (8 tok x 256 x 8 bit), scales  64 B (8 tok x 4 fp16)
+//   F8 part (E4M3):  codes 2048 B (8 tok x 256 x 8 bit), scales  16 B (8 tok x 1 fp16)
+//   F4 part (E2M1):  codes 1024 B (8 tok x 256 x 4 bit), scales 128 B (8 tok x 16 E4M3)
 //
-// Formats: INT8 = (K I8, V I8); Q4_0 = (K Q4, V Q4); K8V4 = (K I8, V Q4).
+// Formats: INT8 = (K I8, V I8); Q4_0 = (K Q4, V Q4); K8V4 = (K I8, V Q4);
+// FP8 = (K F8, V F8); NVFP4 = (K F4, V F4).
 //
 // Code arrangement inside a tile (r = token in tile 0..7).  Each is the
 // register-fragment order of mma.sync.m16n8k16 so that lane (g = lane/4,
@@ -48,14 +51,28 @@ constexpr int WS_TAIL = 16;       // m[8], l[8] after o[G][256] in one workspace
 //  V side, I8: word W(p, m, g) (m-tile m = 16 dims) at
 //      (m>>2)*512 + (g*4 + p)*16 + (m&3)*4; byte n holds token 2p + (n&1),
 //      dim 16m + g + 8(n>>1).
-//  Scales (fp16): Q4 token r, block b at (r>>1)*32 + b*4 + (r&1)*2;
-//                 I8 token r, group q at (r>>1)*16 + q*4 + (r&1)*2.
+//  F8 codes (one byte each) sit where I8 codes would: E4M3 bytes of dims
+//      (2j, 2j+1) and (2j+8, 2j+9) of a k-step, or of tokens (2p, 2p+1) at one
+//      dim, are adjacent, as one cvt.e4m3x2 converts them.
+//  K side, F4: word W(r, b, j) where Q4 puts it; byte q holds the dims
+//      (32b + 2j + 8q', +1) with q' = {0, 1, 2, 3}[q] -> {0, 8, 16, 24}: low
+//      nibble the even dim, high nibble the odd one (one cvt.e2m1x2 per byte).
+//  V side, F4: as Q4 (each token fills its own 16-bit half of a word, so two
+//      tokens of a pair never share a byte and appends never overwrite each
+//      other); the PV warp pairs the nibbles of tokens 2p, 2p+1 itself.
+//  Scales: Q4 (fp16) token r, block b at (r>>1)*32 + b*4 + (r&1)*2;
+//          I8 (fp16) token r, group q at (r>>1)*16 + q*4 + (r&1)*2;
+//          F8 (fp16) token r at 2r;
+//          F4 (E4M3) token r, block b (16 dims) at (r>>1)*32 + b*2 + (r&1).
 // int8 codes are stored as two's complement bytes.
 // ---------------------------------------------------------------------------
-enum Part : int { PART_Q4 = 0, PART_I8 = 1 };
+enum Part : int { PART_Q4 = 0, PART_I8 = 1, PART_F8 = 2, PART_F4 = 3 };
 
-__host__ __device__ constexpr int part_code_bytes(int p) { return p == PART_Q4 ? 1024 : 2048; }
-__host__ __device__ constexpr int part_scale_bytes(int p) { return p == PART_Q4 ? 128 : 64; }
+__host__ __device__ constexpr bool part_nibbles(int p) { return p == PART_Q4 || p == PART_F4; }
+__host__ __device__ constexpr int part_code_bytes(int p) { return part_nibbles(p) ? 1024 : 2048; }
+__host__ __device__ constexpr int part_scale_bytes(int p) {
+    return p == PART_Q4 ? 128 : (p == PART_I8 ? 64 : (p == PART_F8 ? 16 : 128));
+}
 
 template <int FMT> struct Fmt;
 template <> struct Fmt<KVQ_INT8> {
@@ -70,6 +87,14 @@ template <> struct Fmt<KVQ_K8V4> {
     static constexpr int KP = PART_I8, VP = PART_Q4;
     static constexpr bool KROT = false, VROT = true;
 };
+template <> struct Fmt<KVQ_FP8> {
+    static constexpr int KP = PART_F8, VP = PART_F8;
+    static constexpr bool KROT = false, VROT = false;
+};
+template <> struct Fmt<KVQ_NVFP4> {
+    static constexpr int KP = PART_F4, VP = PART_F4;
+    static constexpr bool KROT = false, VROT = false;
+};
 
 template <int FMT> struct TileLayout {
     static constexpr int KP = Fmt<FMT>::KP, VP = Fmt<FMT>::VP;
@@ -81,8 +106,42 @@ template <int FMT> struct TileLayout {
     static constexpr int PAGE_BYTES = BYTES * TILES_PER_PAGE;
 };
 
-inline int host_part_k(int fmt) { return fmt == KVQ_Q4_0 ? PART_Q4 : PART_I8; }
-inline int host_part_v(int fmt) { return fmt == KVQ_INT8 ? PART_I8 : PART_Q4; }
+inline int host_part_k(int fmt) {
+    return fmt == KVQ_Q4_0 ? PART_Q4 : (fmt == KVQ_FP8 ? PART_F8 : (fmt == KVQ_NVFP4 ? PART_F4 : PART_I8));
+}
+inline int host_part_v(int fmt) {
+    return fmt == KVQ_INT8 ? PART_I8 : (fmt == KVQ_FP8 ? PART_F8 : (fmt == KVQ_NVFP4 ? PART_F4 : PART_Q4));
+}
+inline bool host_valid_format(int fmt) { return fmt >= KVQ_INT8 && fmt <= KVQ_NVFP4; }
+inline bool host_rotated_v(int fmt) { return fmt == KVQ_Q4_0 || fmt == KVQ_K8V4; }
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 / FP4 E2M1 conversions (PTX cvt; round to nearest even, and
+// saturating to the largest finite value on the way down).
+// ---------------------------------------------------------------------------
+// Two E4M3 bytes (low byte -> low half) as an exact fp16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v16) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(v16));
+    return r;
+}
+// Two E2M1 nibbles of one byte (low nibble -> low half) as an exact fp16 pair.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t v8) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(v8));
+    return r;
+}
+// One value to E4M3 (the byte) / E2M1 (the nibble).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(x));
+    return r & 0xFFu;
+}
+__device__ __forceinline__ uint32_t f32_to_e2m1(float x) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(r) : "f"(x));
+    return r & 0xFu;
+}
 
 struct PoolGeom {
     int64_t layer_stride, slot_stride, page_bytes;

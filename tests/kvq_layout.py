@@ -9,11 +9,11 @@ import functools
 
 import numpy as np
 
-Q4, I8 = "q4", "i8"
-PARTS = {"int8": (I8, I8), "q4_0": (Q4, Q4), "k8v4": (I8, Q4)}
-CODE_BYTES = {Q4: 1024, I8: 2048}
-SCALE_BYTES = {Q4: 128, I8: 64}
-N_SCALES = {Q4: 8, I8: 4}
+Q4, I8, F8, F4 = "q4", "i8", "f8", "f4"
+PARTS = {"int8": (I8, I8), "q4_0": (Q4, Q4), "k8v4": (I8, Q4), "fp8": (F8, F8), "nvfp4": (F4, F4)}
+CODE_BYTES = {Q4: 1024, I8: 2048, F8: 2048, F4: 1024}
+SCALE_BYTES = {Q4: 128, I8: 64, F8: 16, F4: 128}
+N_SCALES = {Q4: 8, I8: 4, F8: 1, F4: 16}
 
 
 def tile_sections(fmt):
@@ -28,9 +28,24 @@ def tile_sections(fmt):
 @functools.lru_cache(None)
 def code_map(part: str, side: str):
     """(byte offset, bit shift) of the code of (token r in tile, dim d): arrays [8, 256]."""
+    if part == F8:                       # E4M3 bytes where int8 bytes would be
+        return code_map(I8, side)
+    if part == F4 and side == "v":       # E2M1 nibbles where q4_0 nibbles would be
+        return code_map(Q4, side)
     off = np.full((8, 256), -1, np.int64)
     sh = np.zeros((8, 256), np.int64)
-    if part == Q4 and side == "k":
+    if part == F4 and side == "k":
+        # word (r, b, j) at the q4_0 place; byte q: dims 32b + 8q + 2j (low
+        # nibble) and + 1 (high nibble)
+        for r in range(8):
+            for b in range(8):
+                for j in range(4):
+                    for q in range(4):
+                        for h in range(2):
+                            d = 32 * b + 8 * q + 2 * j + h
+                            off[r, d] = (b >> 2) * 512 + (r * 4 + j) * 16 + (b & 3) * 4 + q
+                            sh[r, d] = 4 * h
+    elif part == Q4 and side == "k":
         for r in range(8):
             for b in range(8):
                 for j in range(4):
@@ -70,13 +85,19 @@ def code_map(part: str, side: str):
 
 @functools.lru_cache(None)
 def scale_map(part: str):
-    """byte offset of the fp16 scale of (token r, block q): [8, n_scales]."""
+    """byte offset of the scale of (token r, block q): [8, n_scales] (fp16 for
+    q4 / i8 / f8, one E4M3 byte for f4)."""
     ns = N_SCALES[part]
-    stride = 32 if part == Q4 else 16
     off = np.zeros((8, ns), np.int64)
     for r in range(8):
         for q in range(ns):
-            off[r, q] = (r >> 1) * stride + q * 4 + (r & 1) * 2
+            if part == F8:
+                off[r, q] = 2 * r
+            elif part == F4:
+                off[r, q] = (r >> 1) * 32 + q * 2 + (r & 1)
+            else:
+                stride = 32 if part == Q4 else 16
+                off[r, q] = (r >> 1) * stride + q * 4 + (r & 1) * 2
     return off
 
 
@@ -84,7 +105,7 @@ def _decode_codes(sec: np.ndarray, part: str, side: str) -> np.ndarray:
     """sec: uint8 [n_tiles, code_bytes] -> codes [n_tiles*8, 256] (uint8; int8 as bytes)."""
     off, sh = code_map(part, side)
     raw = sec[:, off]                              # [n_tiles, 8, 256]
-    if part == Q4:
+    if part in (Q4, F4):
         raw = (raw >> sh[None]) & 0xF
     return raw.reshape(-1, 256).astype(np.uint8)
 
@@ -92,6 +113,8 @@ def _decode_codes(sec: np.ndarray, part: str, side: str) -> np.ndarray:
 def _decode_scales(sec: np.ndarray, part: str) -> np.ndarray:
     off = scale_map(part)
     lo = sec[:, off].astype(np.uint16)
+    if part == F4:
+        return lo.reshape(-1, N_SCALES[part])
     hi = sec[:, off + 1].astype(np.uint16)
     return (lo | (hi << 8)).reshape(-1, N_SCALES[part])
 

@@ -21,6 +21,8 @@ SAMPLES = {
     "qwen27b_q4_0_262k": [(0, 0), (0, 2)],
     "ragged4_q4_0": [(0, 1), (2, 2), (3, 3)],
     "ragged4_k8v4": [(1, 0), (2, 3)],
+    "qwen27b_fp8_262k": [(0, 1)],
+    "qwen27b_nvfp4_262k": [(0, 3)],
 }
 
 

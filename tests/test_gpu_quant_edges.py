@@ -80,16 +80,48 @@ def i8_rows():
     return [a, b]
 
 
+def f8_rows():
+    """Vectors that hit the fp8 edge cases (one fp16 scale d per vector)."""
+    a = np.zeros(256, np.float32)
+    a[0] = 448.0                                              # d = 1: codes are the E4M3 of x itself
+    a[1:9] = [2.0 ** -9, 3 * 2.0 ** -10, 2.0 ** -10, -2.0 ** -11, 1.0625, 17.0, -18.0, 232.0]   # subnormals, ties
+    a[9:12] = [-0.0, 1e-30, -1e-30]                           # signed zeros out of underflow
+    b = np.zeros(256, np.float32)                             # all zero: d = 0, codes +0
+    c = np.zeros(256, np.float32)
+    c[5] = np.float32(448.0 * (1 + 0.9 * 2.0 ** -11))         # d rounds down: x / d > 448 saturates
+    c[6] = -c[5]
+    c[7] = 3.0
+    d = (np.arange(256, dtype=np.float32) - 128) * np.float32(0.37)    # a ramp
+    return [a, b, c, d]
+
+
+def f4_rows():
+    """Vectors whose 16-value blocks hit the nvfp4 edge cases (E4M3 scale s per block)."""
+    a = np.zeros(256, np.float32)
+    a[0:8] = [6.0, 0.25, 0.75, 1.25, 2.5, 3.5, 5.0, -5.0]    # s = 1: ties go to the even code
+    a[16:20] = [6.0, -0.0, 7.0, -1.75]                        # s = 1 again; 7 saturates to 6 s
+    # block 2 all zero: s = 0, codes +0
+    a[48:64] = np.float32(0.01)                               # s in the E4M3 subnormal range
+    a[64] = np.float32(6.0 * 448.0 * 1.5)                     # max|x| / 6 above 448: s saturates, codes too
+    a[65] = -1000.0
+    a[80:96] = np.linspace(-3, 3, 16, dtype=np.float32)
+    a[96:112] = np.float32(6.0 * 2.0 ** -12)                  # s underflows to 0
+    b = (np.arange(256, dtype=np.float32) % 17 - 8) * np.float32(0.61)
+    return [a, b]
+
+
+ROWS = {"q4": q4_rows, "i8": i8_rows, "e4m3": f8_rows, "e2m1": f4_rows}
+
+
 def stored_domain(fmt):
     """(K rows, V rows) as the quantiser must see them, and the inputs that
     produce them (rotated parts pass through the inverse transform)."""
-    kq = q4_rows() if fmt == "q4_0" else i8_rows()
-    vq = i8_rows() if fmt == "int8" else q4_rows()
+    kp, vp, k_rot, v_rot = oracle.PARTS[fmt]
+    kq = ROWS[kp]()
+    vq = ROWS[vp]()
     n = max(len(kq), len(vq))
     kq = [kq[i % len(kq)] for i in range(n)]
     vq = [vq[i % len(vq)] for i in range(n)]
-    k_rot = fmt == "q4_0"
-    v_rot = fmt != "int8"
 
     def to_input(y, rot):
         y = np.stack(y)
@@ -118,8 +150,8 @@ def _check_codes(dw, fmt, pos, k_in, v_in, k_seen, v_seen, tag):
     assert np.array_equal(vc[sl], ovc), f"{tag}: V codes"
     assert np.array_equal(vs[sl], ovs), f"{tag}: V scales"
     # the oracle itself on the values the quantiser saw (no rotation involved)
-    quant_k = oracle.quant_q4_0 if fmt == "q4_0" else oracle.quant_int8
-    quant_v = oracle.quant_int8 if fmt == "int8" else oracle.quant_q4_0
+    quant_k = oracle.QUANT[oracle.PARTS[fmt][0]]
+    quant_v = oracle.QUANT[oracle.PARTS[fmt][1]]
     for i in range(len(k_in)):
         c, s = quant_k(k_seen[i])
         assert np.array_equal(okc[i].view(np.uint8), c.view(np.uint8)) and np.array_equal(oks[i], s)
@@ -127,7 +159,7 @@ def _check_codes(dw, fmt, pos, k_in, v_in, k_seen, v_seen, tag):
         assert np.array_equal(ovc[i].view(np.uint8), c.view(np.uint8)) and np.array_equal(ovs[i], s)
 
 
-@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
 def test_kv_append_edge_cases_bit_exact(fmt):
     k_in, v_in, k_seen, v_seen = stored_domain(fmt)
     n = len(k_in)
@@ -146,7 +178,7 @@ def test_kv_append_edge_cases_bit_exact(fmt):
         _check_codes(dw, fmt, pos, k_in, v_in, k_seen, v_seen, f"kv_append/{fmt}/pos={pos}")
 
 
-@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
 def test_decode_step_encodes_edge_cases_bit_exact(fmt):
     """The decode step's own encode of the newest token, one crafted row per
     step, and the step's output against the oracle on the resulting codes."""

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol():
     assert kvq.lib().kvq_version().startswith(b"kvq")
 
 
-@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4"])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
 def test_pool_bytes_match_format_sizes(fmt):
     d = kvq.make_desc(3, 2, 12, 5, fmt)
     L = kvq.pool_layout(d)
@@ -64,14 +64,16 @@ def test_full_window_pool_is_the_printed_size():
     assert two_heads == 1056
 
 
-@pytest.mark.parametrize("part,side", [("q4", "k"), ("q4", "v"), ("i8", "k"), ("i8", "v")])
+@pytest.mark.parametrize("part,side", [(p, s) for p in ("q4", "i8", "f8", "f4") for s in ("k", "v")])
 def test_layout_decoder_is_a_bijection(part, side):
     off, sh = kvq_layout.code_map(part, side)
     keys = off * 8 + sh
     assert len(np.unique(keys)) == 8 * 256
     assert off.max() < kvq_layout.CODE_BYTES[part]
     so = kvq_layout.scale_map(part)
-    assert len(np.unique(so)) == so.size and so.max() + 2 <= kvq_layout.SCALE_BYTES[part]
+    width = 1 if part == "f4" else 2                      # E4M3 byte or fp16 scale
+    cover = np.unique((so[..., None] + np.arange(width)).ravel())
+    assert len(cover) == so.size * width and so.max() + width <= kvq_layout.SCALE_BYTES[part]
 
 
 def _check_plan(plan, info, seq_lens, n_kv, n_ctas):
@@ -142,3 +144,10 @@ def test_validation_errors_without_a_gpu():
                                     info.workspace_bytes, None, None) == -3
     assert L.attn_combine(None, 0x3000, ctypes.byref(info), 1, 0x5000, None, None) == -1
     assert L.paged_decode_attn_cudacore(7, *args, info.workspace_bytes, None, None) == -1
+    # the CUDA-core control decodes the integer-code formats only
+    for f in (kvq.FP8, kvq.NVFP4):
+        assert L.paged_decode_attn_cudacore(f, *args, info.workspace_bytes, None, None) == -2
+    assert L.paged_decode_attn_fp8(*args, info.workspace_bytes, None, None) == -1           # pool is q4_0
+    assert L.paged_decode_attn_nvfp4(*args, info.workspace_bytes, None, None) == -1
+    bad = kvq.make_desc(1, 4, 24, 8, 5)                                                     # no such format
+    assert L.kvq_pool_bytes(ctypes.byref(bad), ctypes.byref(ctypes.c_uint64())) == -1
