@@ -249,7 +249,8 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
-OTHER_WORKLOADS = ("qwen27b_int8_32k", "flashnext_k8v4_128k", "ragged4_q4_0", "ragged4_k8v4")
+OTHER_WORKLOADS = ("qwen27b_int8_32k", "flashnext_k8v4_128k", "ragged4_q4_0", "ragged4_k8v4", "qwen27b_fp8_262k",
+                   "qwen27b_nvfp4_262k")
 
 
 def measure_workload(name: str, layers: int, steps: int, warmup: int, peak: float, uuid: str):
