@@ -338,6 +338,26 @@ int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const f
                                const kvq_plan_info *info, float *workspace, uint64_t workspace_bytes,
                                int32_t *status, void *stream);
 
+/* paged_prefill_attn: chunked-prefill attention over the quantised cache
+ * ([Strata] "能力速览": reading a long prompt is the step before decoding;
+ * "三种 KV 格式横向对比": prompt speed is part of each format's cost).  The
+ * n_tok tokens of sequence seq at positions pos0 .. pos0 + n_tok - 1 must
+ * already be in the pool (kv_append of the chunk; that call already takes
+ * several tokens per sequence).  Each token i attends, per query head, over
+ * the keys 0 .. pos0 + i of the sequence, dequantised from the pool, with the
+ * same softmax scale and output (un-rotated for q4_0 and k8v4) as the decode.
+ *  q        device fp32 [n_tok][n_q_heads][256], prepared as for
+ *           paged_decode_attn (q_rotate'd for q4_0)
+ *  page_table device int32 [n_seq][max_pages]; row seq is used
+ *  out_bf16 device [n_tok][n_q_heads][256] bf16 (required); out_f32 the same
+ *           in fp32 (optional)
+ * Any pool format.  One CTA per 64 (token, head) rows of one KV head reads the
+ * sequence's keys once for all its rows.  KVQ_EINVAL / KVQ_EALIGN on bad
+ * arguments; KVQ_STATUS_* in *status as for the decode. */
+int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq, int pos0, int n_tok,
+                       const int32_t *page_table, int max_pages, int n_seq, uint16_t *out_bf16, float *out_f32,
+                       int32_t *status, void *stream);
+
 /* attn_combine: for each (sequence, query head), merge the partials of its
  * units with the log-sum-exp rule (M = max m_j, L = sum l_j 2^(m_j - M),
  * o' = sum 2^(m_j - M) o_j / L), then, if inverse_fwht is non-zero (q4_0 and

@@ -39,7 +39,7 @@ EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_a
            "paged_decode_attn_fp8_combined", "paged_decode_attn_nvfp4_combined",
            "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine",
            "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4",
-           "paged_decode_step_fp8", "paged_decode_step_nvfp4"]
+           "paged_decode_step_fp8", "paged_decode_step_nvfp4", "paged_prefill_attn"]
 _FMT_NAMES = ("int8", "q4_0", "k8v4", "fp8", "nvfp4")
 
 
@@ -97,6 +97,7 @@ def lib():
             getattr(L, "paged_decode_step_" + f).argtypes = [ctypes.POINTER(Pool), I32, P, P, P, P, I32, P,
                                                              ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P, P, P]
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
+        L.paged_prefill_attn.argtypes = [ctypes.POINTER(Pool), I32, P, I32, I32, I32, P, I32, I32, P, P, P, P]
         for n in EXPORTS[1:]:
             getattr(L, n).restype = ctypes.c_int
         _lib = L
@@ -281,6 +282,18 @@ def paged_decode_attn_fp8(pool, layer, q, page_table, plan_dev, info, workspace,
 def paged_decode_attn_nvfp4(pool, layer, q, page_table, plan_dev, info, workspace, status=None, stream=None):
     assert pool.fmt == NVFP4
     paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
+
+
+def paged_prefill_attn(pool: KVPool, layer: int, q, seq: int, pos0: int, page_table, out_bf16, out_f32=None,
+                       status=None, stream=None):
+    """Chunked-prefill attention: q [n_tok, n_q_heads, 256] (prepared as for
+    the decode) of sequence seq at positions pos0 .. pos0 + n_tok - 1, whose
+    keys are already in the pool, attends causally over the sequence's cache."""
+    cp = pool.c_pool()
+    n_tok = q.shape[0]
+    _check(lib().paged_prefill_attn(ctypes.byref(cp), layer, _ptr(q), seq, pos0, n_tok, _ptr(page_table),
+                                    page_table.shape[1], page_table.shape[0], _ptr(out_bf16), _ptr(out_f32),
+                                    _ptr(status), _stream(stream)), "paged_prefill_attn")
 
 
 def attn_combine(workspace, plan_dev, info: PlanInfo, inverse_fwht: bool, out_bf16, out_f32=None, stream=None):

@@ -322,6 +322,23 @@ KVQ_STEP(paged_decode_step_fp8, KVQ_FP8)
 KVQ_STEP(paged_decode_step_nvfp4, KVQ_NVFP4)
 #undef KVQ_STEP
 
+int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq, int pos0, int n_tok,
+                       const int32_t *page_table, int max_pages, int n_seq, uint16_t *out_bf16, float *out_f32,
+                       int32_t *status, void *stream) {
+    PoolGeom geo;
+    const int rc = check_pool(pool, layer, &geo);
+    if (rc) return rc;
+    if (!q || !page_table || !out_bf16 || n_tok <= 0 || pos0 < 0 || max_pages <= 0 || seq < 0 || seq >= n_seq)
+        return KVQ_EINVAL;
+    if ((int64_t)max_pages * PAGE > INT32_MAX || (int64_t)pos0 + n_tok > (int64_t)max_pages * PAGE) return KVQ_EINVAL;
+    if ((int64_t)n_tok * pool->desc.n_q_heads > ((int64_t)1 << 28)) return KVQ_EINVAL;
+    if (!aligned16(q) || !aligned16(out_bf16) || (out_f32 && !aligned16(out_f32))) return KVQ_EALIGN;
+    return cuda_rc(launch_prefill(pool->desc.fmt, static_cast<const uint8_t *>(pool->base), geo, layer, q, seq, pos0,
+                                  n_tok, page_table, max_pages, pool->desc.n_q_heads,
+                                  host_rotated_v(pool->desc.fmt) ? 1 : 0, out_bf16, out_f32, status,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,
                  uint16_t *out_bf16, float *out_f32, void *stream) {
     if (!workspace || !plan || !info || !out_bf16) return KVQ_EINVAL;

@@ -330,15 +330,16 @@ template <int FMT> struct QkWarp {
     __device__ __forceinline__ uint4 qa(int ks, int lane) const { return lds128(qf + (ks * 32 + lane) * 16); }
 
     // Every QK warp computes the fragments (and its own offset fragment);
-    // `writer` stores them to q_frag.
-    __device__ __forceinline__ void init(const float *qg, int G, int lane, uint8_t *q_frag, bool writer) {
-        const int g = lane >> 2, t = lane & 3;
+    // `writer` stores them to q_frag.  qrow: the query vector of this lane's
+    // row g = lane / 4 (read only when row_ok; otherwise the row is zero).
+    __device__ __forceinline__ void init(const float *qrow, bool row_ok, int lane, uint8_t *q_frag, bool writer) {
+        const int t = lane & 3;
         qf = q_frag;
         float mx = 0.f;
-        if (g < G) {
+        if (row_ok) {
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks) {
-                const float *p = qg + g * D + 16 * ks + 2 * t;
+                const float *p = qrow + 16 * ks + 2 * t;
                 mx = fmaxf(mx, fmaxf(fmaxf(fabsf(p[0] * QSCALE), fabsf(p[1] * QSCALE)),
                                      fmaxf(fabsf(p[8] * QSCALE), fabsf(p[9] * QSCALE))));
             }
@@ -356,8 +357,8 @@ template <int FMT> struct QkWarp {
 #pragma unroll
         for (int ks = 0; ks < 16; ++ks) {
             float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (g < G) {
-                const float *p = qg + g * D + 16 * ks + 2 * t;
+            if (row_ok) {
+                const float *p = qrow + 16 * ks + 2 * t;
                 x[0] = (p[0] * QSCALE) * s_lo; x[1] = (p[1] * QSCALE) * s_lo;
                 x[2] = (p[8] * QSCALE) * s_hi; x[3] = (p[9] * QSCALE) * s_hi;
             }
@@ -538,9 +539,11 @@ template <int FMT> struct QkWarp {
     // rescale factor of head g at [PA + g].  The running max keeps one binade of
     // headroom (it moves to max + 1 only when a score exceeds it), so the rescale
     // factor is rarely different from 1 and p stays <= 1/2 (p' <= 2^(sigma - 1)).
-    template <bool MASK>
+    // lim (CAUSAL only): index, from the item's first token, of the last key
+    // this lane's row may see (a prefill row sees keys up to its own position).
+    template <bool MASK, bool CAUSAL = false>
     __device__ __forceinline__ void item(const uint8_t *tp, const float *fp, const int (&v)[C::TPI], int lane,
-                                         float *slot) {
+                                         float *slot, int lim = 0) {
         constexpr int NS2 = 2 * C::TPI;       // scores per lane: tokens 2t, 2t+1 of each tile
         const int g = lane >> 2, t = lane & 3;
         float s[NS2];
@@ -558,6 +561,13 @@ template <int FMT> struct QkWarp {
                 if (2 * t + 1 >= v[j]) s[2 * j + 1] = -INFINITY;
             }
         }
+        if (CAUSAL) {
+#pragma unroll
+            for (int j = 0; j < C::TPI; ++j) {
+                if (8 * j + 2 * t > lim) s[2 * j] = -INFINITY;
+                if (8 * j + 2 * t + 1 > lim) s[2 * j + 1] = -INFINITY;
+            }
+        }
         float mx = s[0];
 #pragma unroll
         for (int i = 1; i < NS2; ++i) mx = fmaxf(mx, s[i]);
@@ -566,7 +576,9 @@ template <int FMT> struct QkWarp {
         mx *= inv_sb;                                          // log2 units
         vmax = max(vmax, item_v_scale_max<FMT>(tp, lane));
         const float m_true = m_run + sg;
-        const float m_new = mx > m_true ? mx + 1.f : m_true;  // mx is finite: every item has a valid token
+        // mx is finite on the first item (every row sees key 0); later a row may
+        // see none of an item's keys (mx = -inf): nothing moves then
+        const float m_new = mx > m_true ? mx + 1.f : m_true;
         sg = (float)pv_sigma((int)(vmax >> 10));
         const float alpha = ex2(m_run - (m_new - sg));        // 1 when unchanged; 0 on the first item
         l_run *= alpha;
@@ -1591,7 +1603,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         // rotates the raw query on the way, as q_rotate would.
         step_stage_query<STEP && Fmt<FMT>::KROT>(qg, pring, G, pw, C::NQK, lane);
         asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
-        qk.init(pring, G, lane, smem + C::QOFF, pw == 0);
+        qk.init(pring + (lane >> 2) * D, (lane >> 2) < G, lane, smem + C::QOFF, pw == 0);
         asm volatile("bar.sync 2, %0;" ::"r"(C::NQK * 32));
         for (int k = 0;; ++k) {
             const int slot = k % C::DP;
@@ -1709,6 +1721,160 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
         wsu[i] = acc;
     }
     publish_unit<FUSED, NCT>(A, seq, kvh, n_units, &s_last, smem);
+}
+
+// ---------------------------------------------------------------------------
+// Chunked prefill attention over the quantised cache
+// ---------------------------------------------------------------------------
+// A chunk of n_tok new tokens of one sequence at positions pos0 .. pos0 +
+// n_tok - 1 (already appended to the pool) attends, each token over the keys
+// 0 .. its own position.  For one KV head, the chunk's query rows are
+// r = i * G + h (token i, head h of the group); a CTA takes ROWS of them, and
+// each of its NW compute warps takes 8 rows and runs the decode's QK and PV
+// products for them over every item of the key range: the stage ring, the
+// scale conversion and the fragments are the decode's, and each stage is read
+// from HBM once for all ROWS rows (the decode reads it for 6 or 8).
+struct PrefillArgs {
+    DecodeArgs d;            // pool, geometry, layer, page table, status (the copy loop's view)
+    int seq, pos0, n_tok, n_rows;
+};
+
+template <int FMT> struct PfCfg {
+    using L = TileLayout<FMT>;
+    using T = TcCfg<FMT>;
+    static constexpr int NW = 8;                          // compute warps, 8 query rows each
+    static constexpr int ROWS = 8 * NW;
+    static constexpr int COPY_WARP = NW, SCALE_WARP = NW + 1;
+    static constexpr int NTHREADS = (NW + 2) * 32;
+    static constexpr int TPI = T::TPI, IPS = 8 / TPI;
+    static constexpr int STAGE_BYTES = 8 * L::BYTES;
+    static constexpr int NS = (FMT == KVQ_Q4_0 || FMT == KVQ_NVFP4) ? 6 : 4;
+    static constexpr int RING = NS * STAGE_BYTES;
+    static constexpr int OBUF = NW * 8 * T::OSTRIDE * 4;   // the epilogue's rows (after the loop, over the ring)
+    static constexpr int DATA = RING > OBUF ? RING : OBUF;
+    static constexpr int SFOFF = (DATA + 127) & ~127;
+    static constexpr int QOFF = SFOFF + NS * T::SF_STAGE_BYTES;      // per warp: 16 k-steps x 32 lanes x 16 B
+    static constexpr int POFF = QOFF + NW * 16 * 32 * 16;            // per warp: one p slot
+    static constexpr int BAR_OFF = (POFF + NW * T::PSLOT * 4 + 15) & ~15;
+    static constexpr int TOTAL = BAR_OFF + 3 * NS * 8 + NS * 4;      // full, ready, empty; stage_ok
+    static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(const __grid_constant__ PrefillArgs P) {
+    using L = TileLayout<FMT>;
+    using C = PfCfg<FMT>;
+    using T = TcCfg<FMT>;
+    const DecodeArgs &A = P.d;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *ready = full + C::NS;
+    uint64_t *empty = ready + C::NS;
+    int *stage_ok = reinterpret_cast<int *>(empty + C::NS);
+
+    grid_dependency_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvh = blockIdx.y, G = A.G;
+    const int r0 = blockIdx.x * C::ROWS;
+    if (r0 >= P.n_rows) return;
+    // keys 0 .. pos0 + (last token of the CTA's rows)
+    const int i_last = min(P.n_tok - 1, (r0 + C::ROWS - 1) / G);
+    const int t_end = P.pos0 + i_last + 1;
+    const int n_steps = (t_end + STEP_TOKENS - 1) / STEP_TOKENS;
+    const int n_items = (t_end + C::TPI * TILE - 1) / (C::TPI * TILE);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&ready[i], 32);
+            mbar_init(&empty[i], 32 * C::NW * C::IPS);     // every compute warp, every item of the stage
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == C::COPY_WARP) {
+        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, P.seq, kvh, 0, n_steps, lane);
+        return;
+    }
+    if (warp == C::SCALE_WARP) {
+        for (int i = 0; i < n_steps; ++i) {
+            const int si = i % C::NS;
+            if (!mbar_wait_bounded(&full[si], (i / C::NS) & 1, WAIT_LIMIT_NS)) {
+                if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+                break;
+            }
+            if (stage_ok[si])
+                convert_stage_scales<FMT>(smem + si * C::STAGE_BYTES,
+                                          reinterpret_cast<float *>(smem + C::SFOFF + si * T::SF_STAGE_BYTES), lane);
+            __syncwarp();
+            mbar_arrive(&ready[si]);
+        }
+        return;
+    }
+
+    // compute warp: rows r0 + 8 warp + g, g = lane / 4
+    const int r = r0 + 8 * warp + (lane >> 2);
+    const bool row_ok = r < P.n_rows;
+    const int tok_i = row_ok ? r / G : 0, head = row_ok ? r % G : 0;
+    const int lim = row_ok ? P.pos0 + tok_i : t_end - 1;        // last key the row sees
+    const float *qrow = A.q + ((int64_t)tok_i * A.n_q_heads + (int64_t)kvh * G + head) * D;
+    QkWarp<FMT> qk;
+    PvWarp<FMT> pv;
+    qk.init(qrow, row_ok, lane, smem + C::QOFF + warp * (16 * 32 * 16), true);
+    __syncwarp();
+    pv.init();
+    float *ps = reinterpret_cast<float *>(smem + C::POFF) + warp * T::PSLOT;
+    for (int it = 0; it < n_items; ++it) {
+        const int st = it / C::IPS, si = st % C::NS, within = it % C::IPS;
+        if (!mbar_wait_bounded(&ready[si], (st / C::NS) & 1, WAIT_LIMIT_NS)) {
+            if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
+            break;
+        }
+        const int tok = it * C::TPI * TILE;
+        int v[C::TPI];
+#pragma unroll
+        for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t_end - tok - j * TILE));
+        const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
+        const bool ok = stage_ok[si] != 0;
+        if (ok) {
+            const float *fp = reinterpret_cast<const float *>(smem + C::SFOFF + si * T::SF_STAGE_BYTES) +
+                              within * C::TPI * T::SF_TILE;
+            if (v[C::TPI - 1] == TILE) qk.template item<false, true>(tp, fp, v, lane, ps, lim - tok);
+            else qk.template item<true, true>(tp, fp, v, lane, ps, lim - tok);
+        } else {
+            qk.skip(lane, ps);
+        }
+        __syncwarp();
+        float4 pp[C::TPI / 2];
+#pragma unroll
+        for (int h = 0; h < C::TPI / 2; ++h) pp[h] = lds128f(ps + lane * 2 * C::TPI + 4 * h);
+        const float2 al = make_float2(ps[T::PA + 2 * (lane & 3)], ps[T::PA + 2 * (lane & 3) + 1]);
+        if (v[C::TPI - 1] == TILE) pv.template item<false>(tp, v, ok, lane, pp, al);
+        else pv.template item<true>(tp, v, ok, lane, pp, al);
+        __syncwarp();                               // the slot is rewritten by the next item
+        mbar_arrive(&empty[si]);
+    }
+
+    // ---- epilogue: o / l per row, un-rotated where the format rotates V ----
+    asm volatile("bar.sync 1, %0;" ::"r"(C::NW * 32));   // every warp is done with the ring
+    float lr = qk.l_run;
+    lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+    lr += __shfl_xor_sync(0xffffffffu, lr, 2);            // row g's sum on lanes 4g .. 4g+3
+    const int t = lane & 3;
+    const float l0 = __shfl_sync(0xffffffffu, lr, 8 * t), l1 = __shfl_sync(0xffffffffu, lr, 8 * t + 4);
+    float *b = reinterpret_cast<float *>(smem) + warp * 8 * T::OSTRIDE;
+    pv.store_scaled(b, l0 > 0.f ? 1.f / l0 : 0.f, l1 > 0.f ? 1.f / l1 : 0.f, lane);
+    __syncwarp();
+    for (int h = 0; h < 8; ++h) {
+        const int rr = r0 + 8 * warp + h;
+        if (rr >= P.n_rows) break;
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = b[h * T::OSTRIDE + lane * 8 + i];
+        const int ti = rr / G, hh = rr % G;
+        finish_row(x, lane, A.inverse_fwht, (int64_t)ti * A.n_q_heads + (int64_t)kvh * G + hh, A.out_bf16, A.out_f32);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1904,6 +2070,46 @@ cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const
                  status, inverse_fwht, out_bf16, out_f32, 0, k_new, v_new};
     if (out_bf16) return launch_fused<true>(fmt, tensor_cores, a, info.n_units, s);
     return launch_fused<false>(fmt, tensor_cores, a, info.n_units, s);
+}
+
+template <int FMT>
+cudaError_t launch_prefill_fmt(const PrefillArgs &p, cudaStream_t s) {
+    using C = PfCfg<FMT>;
+    static std::mutex mu;
+    static bool configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev]) {
+            cudaError_t e =
+                cudaFuncSetAttribute(prefill_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::TOTAL);
+            if (e != cudaSuccess) return e;
+            configured[dev] = true;
+        }
+    }
+    const dim3 grid((unsigned)((p.n_rows + C::ROWS - 1) / C::ROWS), (unsigned)p.d.geo.n_kv_heads);
+    return launch_ex(prefill_tc_kernel<FMT>, grid, dim3(C::NTHREADS), C::TOTAL, s, false, p);
+}
+
+cudaError_t launch_prefill(int fmt, const uint8_t *pool, const PoolGeom &geo, int layer, const float *q, int seq,
+                           int pos0, int n_tok, const int32_t *page_table, int max_pages, int n_q_heads,
+                           int inverse_fwht, uint16_t *out_bf16, float *out_f32, int32_t *status, cudaStream_t s) {
+    const int G = n_q_heads / geo.n_kv_heads;
+    PrefillArgs p{};
+    p.d = DecodeArgs{pool, geo, layer, q, page_table, max_pages, nullptr, n_q_heads, G, nullptr,
+                     status, inverse_fwht, out_bf16, out_f32, 0, nullptr, nullptr};
+    p.seq = seq;
+    p.pos0 = pos0;
+    p.n_tok = n_tok;
+    p.n_rows = n_tok * G;
+    switch (fmt) {
+    case KVQ_INT8: return launch_prefill_fmt<KVQ_INT8>(p, s);
+    case KVQ_Q4_0: return launch_prefill_fmt<KVQ_Q4_0>(p, s);
+    case KVQ_K8V4: return launch_prefill_fmt<KVQ_K8V4>(p, s);
+    case KVQ_FP8: return launch_prefill_fmt<KVQ_FP8>(p, s);
+    default: return launch_prefill_fmt<KVQ_NVFP4>(p, s);
+    }
 }
 
 cudaError_t launch_combine(const float *ws, const int32_t *plan, const kvq_plan_info &info, int inverse_fwht,

@@ -343,6 +343,9 @@ cudaError_t launch_append_rotate(int fmt, uint8_t *pool, const PoolGeom &geo, in
                                  const float *v, int64_t n_rows, const int32_t *row_seq, const int32_t *row_pos,
                                  const int32_t *page_table, int max_pages, int n_seq, int32_t *status, const float *q,
                                  float *q_rot, int64_t n_vec, cudaStream_t s);
+cudaError_t launch_prefill(int fmt, const uint8_t *pool, const PoolGeom &geo, int layer, const float *q, int seq,
+                           int pos0, int n_tok, const int32_t *page_table, int max_pages, int n_q_heads,
+                           int inverse_fwht, uint16_t *out_bf16, float *out_f32, int32_t *status, cudaStream_t s);
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
                           const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht,
