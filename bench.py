@@ -37,12 +37,23 @@ DEFAULT_WORKLOAD = "qwen27b_q4_0_262k"
 FALLBACK_HBM_GBS = 6650.0
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense fp16/bf16 tensor throughput to hold a kernel timed on its own against (burst)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured cuBLAS bf16 GEMM (burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback 1.59 PFLOP/s"
 
 
 def decode_source_hash() -> str:
@@ -251,6 +262,54 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 OTHER_WORKLOADS = ("qwen27b_int8_32k", "flashnext_k8v4_128k", "ragged4_q4_0", "ragged4_k8v4", "qwen27b_fp8_262k",
                    "qwen27b_nvfp4_262k")
+
+
+def measure_prefill(T: int, n_tok: int, steps: int, warmup: int, uuid: str):
+    """paged_prefill_attn of the last n_tok tokens of a T-token sequence on one
+    layer of the 27B q4_0 shape (24 Q / 4 KV heads), timed with CUDA events
+    over `steps` calls; useful FLOPs = 4 x 256 per (query row, key) pair in the
+    causal range (QK and PV, 2 per multiply-add).  Returns a sub-record."""
+    import torch
+    import kvq_inputs
+    import quantized_kv_cache_17_b200 as kvq
+    from kvq_inputs import device as kdev
+    w = kvq_inputs.Workload(name=f"prefill_q4_0_{T // 1024}k_{n_tok}", index=4, fmt="q4_0", n_layers=1,
+                            n_q_heads=24, n_kv_heads=4, seq_lens=[T], page_order="contiguous", n_outlier=8,
+                            outlier_kind="student_t", q_post=1.0 / 16, q_outliers=False)
+    dw = kdev.build_pool(w, prefill_last=True)
+    qt = kdev.DeviceTable(w.q_table(0), "cuda")
+    qp = kvq.q_rotate(kdev.gen_rows_device(w.q_key(0, 0), qt, 0, n_tok))
+    out_bf = torch.empty((n_tok, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pos0 = T - n_tok
+    for _ in range(warmup):
+        kvq.paged_prefill_attn(dw.pool, 0, qp, 0, pos0, dw.page_table, out_bf, status=status)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    a.record(stream)
+    for _ in range(steps):
+        kvq.paged_prefill_attn(dw.pool, 0, qp, 0, pos0, dw.page_table, out_bf, status=status)
+    b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    assert int(status.item()) == 0, f"kernel status {status.item()} in the prefill"
+    us = a.elapsed_time(b) * 1e3 / steps
+    keys = float(np.arange(pos0 + 1, T + 1, dtype=np.float64).sum())
+    flops = 4.0 * 256 * w.n_q_heads * keys
+    tpk, tsrc = tensor_peak()
+    tflops = flops / (us * 1e-6) / 1e12
+    rec = {"workload": w.name, "format": "q4_0", "context": T, "chunk_tokens": n_tok, "us_per_layer": round(us, 1),
+           "useful_tflops": round(tflops, 2), "tok_s_16_layers": round(n_tok / (16 * us * 1e-6), 1),
+           "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": tpk, "unit": "TFLOP/s",
+                        "frac": round(tflops / tpk, 4), "peak_source": tsrc},
+           "clocks": clocks}
+    del dw, qp, out_bf
+    torch.cuda.empty_cache()
+    return rec
 
 
 def measure_workload(name: str, layers: int, steps: int, warmup: int, peak: float, uuid: str):
@@ -562,11 +621,13 @@ def run_ours(args):
                          f"encode of one token per KV head and layer, single thread"}
 
     others = None
+    prefill = None
     if rank == 0 and world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD and not use_alu \
             and not args.layers:
         del dw, q, k_new, v_new, ws, out_bf, out_f, q_rot
         torch.cuda.empty_cache()
         others = [measure_workload(n, args.other_layers, args.steps, args.warmup, peak, uuid) for n in OTHER_WORKLOADS]
+        prefill = measure_prefill(32768, 512, max(2, args.steps // 4), args.warmup, uuid)
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -598,7 +659,8 @@ def run_ours(args):
                 "launch": "CUDA graph of the 16-layer step",
                 "clocks": clocks,
                 "cpu_baseline": cpu,
-                "other_workloads": others}
+                "other_workloads": others,
+                "prefill": prefill}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
