@@ -312,6 +312,85 @@ def measure_prefill(T: int, n_tok: int, steps: int, warmup: int, uuid: str):
     return rec
 
 
+def measure_resident(T: int, steps: int, warmup: int, uuid: str):
+    """Host-resident KV: one layer of the 27B q4_0 shape at T tokens kept in a
+    pinned host pool, paged into a device cache by kvq_resident_load (the
+    zero-copy page-in kernel), timed with CUDA events; beside it the copy engine
+    moving the same bytes in one cudaMemcpyAsync (the bus ceiling), the host
+    planning time of kvq_resident_map for an all-miss and an all-hit call, and a
+    cold layer (page-in of every page, then the decode).  Returns a sub-record."""
+    import torch
+    import kvq_inputs
+    import quantized_kv_cache_17_b200 as kvq
+    from kvq_inputs import device as kdev
+    w = kvq_inputs.Workload(name=f"resident_q4_0_{T // 1024}k", index=4, fmt="q4_0", n_layers=1, n_q_heads=24,
+                            n_kv_heads=4, seq_lens=[T], page_order="permuted", n_outlier=8,
+                            outlier_kind="student_t", q_post=1.0 / 16, q_outliers=False)
+    dw = kdev.build_pool(w)
+    H = kvq.KVPool.allocate(dw.pool.desc, "pinned")
+    H.buf.copy_(dw.pool.buf)
+    n_pages = dw.pool.desc.n_pages
+    dw.pool = None
+    torch.cuda.empty_cache()
+    C = kvq.KVPool.allocate(kvq.make_desc(1, w.n_kv_heads, w.n_q_heads, n_pages, "q4_0"))
+    rc = kvq.ResidentCache(H, C)
+    t0 = time.perf_counter()
+    cpt, loads = rc.map(0, dw.page_table_host, w.seq_lens)
+    map_miss_us = (time.perf_counter() - t0) * 1e6
+    t0 = time.perf_counter()
+    for _ in range(20):
+        rc.map(0, dw.page_table_host, w.seq_lens)
+    map_hit_us = (time.perf_counter() - t0) * 1e6 / 20
+    nbytes = len(loads) * kvq.pool_layout(C.desc).slot_stride
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(warmup):
+        rc.load(0, loads)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    ev[0].record(stream)
+    for _ in range(steps):
+        rc.load(0, loads)
+    ev[1].record(stream)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dst.copy_(H.buf[:nbytes], non_blocking=True)
+    ev[2].record(stream)
+    for _ in range(steps):
+        dst.copy_(H.buf[:nbytes], non_blocking=True)
+    ev[3].record(stream)
+    # cold layer: page every page in, then decode over the cache
+    cpt_d = torch.from_numpy(cpt).cuda()
+    plan, info = kvq.decode_plan(C.desc, w.seq_lens, cpt.shape[1])
+    plan_d = torch.from_numpy(plan).cuda()
+    ws = torch.zeros(info.workspace_bytes // 4, dtype=torch.float32, device="cuda")
+    qt = kdev.DeviceTable(w.q_table(0), "cuda")
+    qp = kvq.q_rotate(kdev.gen_rows_device(w.q_key(0, 0), qt, 0, 1))
+    out_bf = torch.empty((1, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ev[4].record(stream)
+    for _ in range(steps):
+        rc.load(0, loads)
+        kvq.paged_decode_attn_combined(C, 0, qp, cpt_d, plan_d, info, ws, out_bf, status=status)
+    ev[5].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    assert int(status.item()) == 0, f"kernel status {status.item()} in the resident decode"
+    load_us = ev[0].elapsed_time(ev[1]) * 1e3 / steps
+    copy_us = ev[2].elapsed_time(ev[3]) * 1e3 / steps
+    cold_us = ev[4].elapsed_time(ev[5]) * 1e3 / steps
+    rec = {"workload": w.name, "format": "q4_0", "context": T, "pages": len(loads), "page_bytes": nbytes // len(loads),
+           "page_in_us": round(load_us, 1), "page_in_gbs": round(nbytes / load_us / 1e3, 2),
+           "copy_engine_gbs": round(nbytes / copy_us / 1e3, 2),
+           "page_in_vs_copy_engine": round(copy_us / load_us, 3),
+           "cold_layer_us": round(cold_us, 1), "map_all_miss_us": round(map_miss_us, 1),
+           "map_all_hit_us": round(map_hit_us, 1), "clocks": clocks}
+    del H, C, rc, dst, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 def measure_workload(name: str, layers: int, steps: int, warmup: int, peak: float, uuid: str):
     """One decode step per layer (paged_decode_step, the bench's timed kernel)
     of workload `name` restricted to its first `layers` layers, captured as a
@@ -622,12 +701,14 @@ def run_ours(args):
 
     others = None
     prefill = None
+    resident = None
     if rank == 0 and world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD and not use_alu \
             and not args.layers:
         del dw, q, k_new, v_new, ws, out_bf, out_f, q_rot
         torch.cuda.empty_cache()
         others = [measure_workload(n, args.other_layers, args.steps, args.warmup, peak, uuid) for n in OTHER_WORKLOADS]
         prefill = measure_prefill(32768, 512, max(2, args.steps // 4), args.warmup, uuid)
+        resident = measure_resident(131072, max(2, args.steps // 4), args.warmup, uuid)
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -660,7 +741,8 @@ def run_ours(args):
                 "clocks": clocks,
                 "cpu_baseline": cpu,
                 "other_workloads": others,
-                "prefill": prefill}
+                "prefill": prefill,
+                "resident": resident}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

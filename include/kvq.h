@@ -368,6 +368,77 @@ int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq,
 int attn_combine(const float *workspace, const int32_t *plan, const kvq_plan_info *info, int inverse_fwht,
                  uint16_t *out_bf16, float *out_f32, void *stream);
 
+/* Host-resident KV with a device page cache ([Strata] "KV 从显存搬进内存之后发生了
+ * 什么": the authoritative copy of the KV cache sits in pinned host memory, the
+ * GPU holds only the pages attention is about to read, a residency table with
+ * CLOCK (second chance) eviction chooses them, missing pages are pulled over the
+ * bus without a staging copy, and attention runs unchanged on the cached pages,
+ * so its output is bit-identical to attention over a fully resident pool).
+ *
+ * host pool : a kvq_pool whose base is pinned, device-mapped host memory
+ *             (cudaHostAlloc / cudaMallocHost; under unified addressing the
+ *             device reaches it directly).  kv_append writes it like any pool.
+ * cache pool: a device kvq_pool with n_layers = 1 and the same format and
+ *             heads; its n_pages are the cache slots.  A slot holds one page
+ *             (every KV head) of any layer.
+ * state     : caller-owned host memory of kvq_resident_state_bytes() bytes
+ *             (header, one record per slot, and a residency table with one
+ *             entry per (layer, host page)); the library allocates nothing.
+ *
+ * Per decode step and layer: kvq_resident_map (host only) turns the host page
+ * table into a cache page table and a list of pages to load; kvq_resident_load
+ * enqueues the page-in; kv_append writes the new token into both pools (the same
+ * kernel on the same input writes the same bytes, so the cached page stays equal
+ * to the host page); the attention entry points then take the cache pool, layer
+ * 0 and the cache page table.  The state is not thread-safe. */
+uint64_t kvq_resident_state_bytes(int n_layers, int n_host_pages, int n_cache_slots);
+
+/* Initialise the state for a host pool and a cache pool (both stay owned by the
+ * caller and must outlive the state).  Every slot starts empty.  KVQ_EINVAL on
+ * mismatched descriptors or a cache pool with n_layers != 1, KVQ_ESIZE if
+ * state_bytes is too small, KVQ_EALIGN if a base is not 16-byte aligned.
+ * Host only; no CUDA call. */
+int kvq_resident_init(void *state, uint64_t state_bytes, const kvq_pool *host_pool, const kvq_pool *cache_pool);
+
+/* Make resident, for layer `layer`, every page the n_seq sequences read:
+ * pages 0 .. ceil(seq_len[b] / 256) - 1 of row b of host_page_table (host int32
+ * [n_seq][max_pages], host page indices).  Writes cache_page_table (host int32
+ * [n_seq][max_pages], slot indices, -1 past each sequence's pages) and, in
+ * loads (host int32 [loads_capacity][2]), the (host page, slot) pairs that
+ * kvq_resident_load must copy, *n_loads of them.
+ * Policy: the distinct pages of the call form its batch.  Resident pages of the
+ * batch get their reference bit set and are pinned for the call.  Each missing
+ * page, in order of first reference (sequence by sequence, page by page), takes
+ * the slot the CLOCK hand finds: the hand skips pinned slots, clears a set
+ * reference bit and moves on, and stops at the first unpinned slot with a clear
+ * bit; the page evicted from it (if any) leaves the table, the new page takes
+ * the slot with its bit set and pinned, and the hand moves one past it.
+ * Statistics count one hit or miss per page reference.
+ * KVQ_EINVAL on a bad argument (the state is unchanged); KVQ_ESIZE, with the
+ * state unchanged, if the batch has more pages than the cache has slots or if
+ * loads_capacity is below the number of missing pages (*n_loads then holds
+ * that number; loads may be NULL with loads_capacity 0 to ask for it).
+ * Host only; no CUDA call. */
+int kvq_resident_map(void *state, int layer, const int32_t *host_page_table, int n_seq, int max_pages,
+                     const int32_t *seq_len, int32_t *cache_page_table, int32_t *loads, int loads_capacity,
+                     int *n_loads);
+
+/* Enqueue on `stream` the copy of each listed page of layer `layer` from the
+ * host pool into its cache slot: one kernel reads the pinned host memory
+ * directly (zero-copy) and writes the slot.  loads is host memory, read before
+ * the call returns (the list travels in the launch parameters, so the caller may
+ * reuse the array at once).  The host pool must not be written between the
+ * map and the completion of this copy except by stream-ordered work.
+ * KVQ_EINVAL on a bad argument or a host pool that is not device-mapped host
+ * memory; KVQ_ECUDA on a launch error. */
+int kvq_resident_load(void *state, int layer, const int32_t *loads, int n_loads, void *stream);
+
+/* The slot holding (layer, host_page), or -1 in *slot.  Host only. */
+int kvq_resident_query(const void *state, int layer, int host_page, int *slot);
+
+/* Hit, miss and eviction counts since init (any pointer may be NULL).  Host only. */
+int kvq_resident_stats(const void *state, int64_t *hits, int64_t *misses, int64_t *evictions);
+
 /* Library version string. */
 const char *kvq_version(void);
 

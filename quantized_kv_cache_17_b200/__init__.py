@@ -39,7 +39,9 @@ EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_a
            "paged_decode_attn_fp8_combined", "paged_decode_attn_nvfp4_combined",
            "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine",
            "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4",
-           "paged_decode_step_fp8", "paged_decode_step_nvfp4", "paged_prefill_attn"]
+           "paged_decode_step_fp8", "paged_decode_step_nvfp4", "paged_prefill_attn",
+           "kvq_resident_state_bytes", "kvq_resident_init", "kvq_resident_map", "kvq_resident_load",
+           "kvq_resident_query", "kvq_resident_stats"]
 _FMT_NAMES = ("int8", "q4_0", "k8v4", "fp8", "nvfp4")
 
 
@@ -98,8 +100,15 @@ def lib():
                                                              ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P, P, P]
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
         L.paged_prefill_attn.argtypes = [ctypes.POINTER(Pool), I32, P, I32, I32, I32, P, I32, I32, P, P, P, P]
+        L.kvq_resident_init.argtypes = [P, ctypes.c_uint64, ctypes.POINTER(Pool), ctypes.POINTER(Pool)]
+        L.kvq_resident_map.argtypes = [P, I32, P, I32, I32, P, P, P, I32, ctypes.POINTER(ctypes.c_int)]
+        L.kvq_resident_load.argtypes = [P, I32, P, I32, P]
+        L.kvq_resident_query.argtypes = [P, I32, I32, ctypes.POINTER(ctypes.c_int)]
+        L.kvq_resident_stats.argtypes = [P] + [ctypes.POINTER(ctypes.c_int64)] * 3
         for n in EXPORTS[1:]:
             getattr(L, n).restype = ctypes.c_int
+        L.kvq_resident_state_bytes.argtypes = [I32, I32, I32]
+        L.kvq_resident_state_bytes.restype = ctypes.c_uint64
         _lib = L
     return _lib
 
@@ -145,7 +154,10 @@ class KVPool:
 
     @staticmethod
     def allocate(desc: PoolDesc, device="cuda"):
+        """device="pinned" gives a pool in pinned, device-mapped host memory."""
         import torch
+        if device == "pinned":
+            return KVPool(desc, torch.zeros(pool_bytes(desc), dtype=torch.uint8).pin_memory())
         return KVPool(desc, torch.zeros(pool_bytes(desc), dtype=torch.uint8, device=device))
 
     def c_pool(self) -> Pool:
@@ -310,3 +322,56 @@ def rotated_v(fmt) -> bool:
 def rotated_q(fmt) -> bool:
     f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
     return f == Q4_0
+
+
+class ResidentCache:
+    """Host-resident KV with a device page cache: the state of the residency
+    table and CLOCK hand (host memory owned here), over a pinned host pool and a
+    one-layer device cache pool that the caller owns."""
+
+    def __init__(self, host_pool: KVPool, cache_pool: KVPool = None, *, host_desc: PoolDesc = None,
+                 cache_desc: PoolDesc = None, host_base: int = None, cache_base: int = None):
+        # host_desc/cache_desc with raw base addresses: planning only (no pool memory behind them)
+        if host_pool is not None:
+            host_desc, host_base = host_pool.desc, host_pool.buf.data_ptr()
+            cache_desc, cache_base = cache_pool.desc, cache_pool.buf.data_ptr()
+        self.host_desc, self.cache_desc = host_desc, cache_desc
+        n = lib().kvq_resident_state_bytes(host_desc.n_layers, host_desc.n_pages, cache_desc.n_pages)
+        if n == 0:
+            raise KVQError("kvq_resident_state_bytes failed: KVQ_EINVAL")
+        self._state = np.zeros((n + 7) // 8, np.uint64)
+        self.state = self._state.ctypes.data
+        hp, cp = Pool(host_base, host_desc), Pool(cache_base, cache_desc)
+        _check(lib().kvq_resident_init(self.state, self._state.nbytes, ctypes.byref(hp), ctypes.byref(cp)),
+               "kvq_resident_init")
+
+    def map(self, layer: int, host_page_table, seq_lens):
+        """Host planning: returns (cache_page_table, loads) as int32 numpy
+        arrays ([n_seq, max_pages] and [n_loads, 2] of (host page, slot))."""
+        hpt = np.ascontiguousarray(np.asarray(host_page_table, np.int32))
+        sl = np.ascontiguousarray(np.asarray(seq_lens, np.int32))
+        n_seq, max_pages = hpt.shape
+        cpt = np.empty_like(hpt)
+        loads = np.empty((self.cache_desc.n_pages, 2), np.int32)
+        nl = ctypes.c_int()
+        _check(lib().kvq_resident_map(self.state, layer, hpt.ctypes.data, n_seq, max_pages, sl.ctypes.data,
+                                      cpt.ctypes.data, loads.ctypes.data, len(loads), ctypes.byref(nl)),
+               "kvq_resident_map")
+        return cpt, loads[:nl.value].copy()
+
+    def load(self, layer: int, loads, stream=None):
+        """Enqueue the page-in of the (host page, slot) pairs in loads."""
+        ld = np.ascontiguousarray(np.asarray(loads, np.int32).reshape(-1, 2))
+        _check(lib().kvq_resident_load(self.state, layer, ld.ctypes.data if len(ld) else None, len(ld),
+                                       _stream(stream)), "kvq_resident_load")
+
+    def slot_of(self, layer: int, host_page: int) -> int:
+        s = ctypes.c_int()
+        _check(lib().kvq_resident_query(self.state, layer, host_page, ctypes.byref(s)), "kvq_resident_query")
+        return s.value
+
+    def stats(self):
+        """(hits, misses, evictions) since construction."""
+        v = [ctypes.c_int64() for _ in range(3)]
+        _check(lib().kvq_resident_stats(self.state, *[ctypes.byref(x) for x in v]), "kvq_resident_stats")
+        return tuple(x.value for x in v)

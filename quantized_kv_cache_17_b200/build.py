@@ -31,6 +31,7 @@ SOURCES = {
     "kvq_append.cu": ["-fmad=false"],     # quantiser: no fused multiply-add anywhere in this unit
     "kvq_decode.cu": [],
     "kvq_noalloc.cu": [],
+    "kvq_resident.cu": [],
 }
 
 
