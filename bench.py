@@ -282,32 +282,46 @@ def measure_prefill(T: int, n_tok: int, steps: int, warmup: int, uuid: str):
     out_bf = torch.empty((n_tok, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     pos0 = T - n_tok
+    n_split, wb = kvq.prefill_split(dw.pool.desc, pos0, n_tok)
+    ws = torch.empty(max(wb, 16) // 4, dtype=torch.float32, device="cuda")
+
+    def run(ns):
+        kvq.paged_prefill_attn(dw.pool, 0, qp, 0, pos0, dw.page_table, out_bf, status=status, n_split=ns,
+                               workspace=ws if ns > 1 else None)
+
     for _ in range(warmup):
-        kvq.paged_prefill_attn(dw.pool, 0, qp, 0, pos0, dw.page_table, out_bf, status=status)
+        run(n_split)
+        run(1)
     torch.cuda.synchronize()
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     stream = torch.cuda.current_stream()
-    a.record(stream)
+    ev[0].record(stream)
     for _ in range(steps):
-        kvq.paged_prefill_attn(dw.pool, 0, qp, 0, pos0, dw.page_table, out_bf, status=status)
-    b.record(stream)
+        run(n_split)
+    ev[1].record(stream)
+    ev[2].record(stream)
+    for _ in range(steps):
+        run(1)
+    ev[3].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     assert int(status.item()) == 0, f"kernel status {status.item()} in the prefill"
-    us = a.elapsed_time(b) * 1e3 / steps
+    us = ev[0].elapsed_time(ev[1]) * 1e3 / steps
+    us_one = ev[2].elapsed_time(ev[3]) * 1e3 / steps
     keys = float(np.arange(pos0 + 1, T + 1, dtype=np.float64).sum())
     flops = 4.0 * 256 * w.n_q_heads * keys
     tpk, tsrc = tensor_peak()
     tflops = flops / (us * 1e-6) / 1e12
     rec = {"workload": w.name, "format": "q4_0", "context": T, "chunk_tokens": n_tok, "us_per_layer": round(us, 1),
+           "n_split": n_split, "us_per_layer_unsplit": round(us_one, 1),
            "useful_tflops": round(tflops, 2), "tok_s_16_layers": round(n_tok / (16 * us * 1e-6), 1),
            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": tpk, "unit": "TFLOP/s",
                         "frac": round(tflops / tpk, 4), "peak_source": tsrc},
            "clocks": clocks}
-    del dw, qp, out_bf
+    del dw, qp, out_bf, ws
     torch.cuda.empty_cache()
     return rec
 

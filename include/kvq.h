@@ -351,12 +351,28 @@ int paged_decode_attn_cudacore(int fmt, const kvq_pool *pool, int layer, const f
  *  page_table device int32 [n_seq][max_pages]; row seq is used
  *  out_bf16 device [n_tok][n_q_heads][256] bf16 (required); out_f32 the same
  *           in fp32 (optional)
- * Any pool format.  One CTA per 64 (token, head) rows of one KV head reads the
- * sequence's keys once for all its rows.  KVQ_EINVAL / KVQ_EALIGN on bad
- * arguments; KVQ_STATUS_* in *status as for the decode. */
+ *  n_split  1: one pass over the keys, results written directly.  2 .. 8: the
+ *           key range is cut into n_split parts (cuts at multiples of 64 tokens,
+ *           all at or below pos0), each part runs as its own CTAs and writes an
+ *           unnormalised partial to workspace, and a second kernel merges the
+ *           parts with the log-sum-exp rule before the output rotation; this
+ *           fills the GPU when the chunk alone gives too few CTAs.
+ *  workspace device fp32, at least the kvq_prefill_split bytes for n_split
+ *           (NULL when n_split is 1); caller-owned, needs no initialisation
+ * Any pool format.  One CTA per 64 (token, head) rows of one KV head (and part)
+ * reads that range of the sequence's keys once for all its rows.  KVQ_EINVAL /
+ * KVQ_EALIGN on bad arguments (also an n_split with no valid cut), KVQ_ESIZE if
+ * the workspace is too small; KVQ_STATUS_* in *status as for the decode. */
 int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq, int pos0, int n_tok,
-                       const int32_t *page_table, int max_pages, int n_seq, uint16_t *out_bf16, float *out_f32,
-                       int32_t *status, void *stream);
+                       const int32_t *page_table, int max_pages, int n_seq, int n_split, float *workspace,
+                       uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status, void *stream);
+
+/* The key-range split paged_prefill_attn should use for a chunk of n_tok tokens
+ * at pos0 on a GPU with n_sms multiprocessors (0: the 148 of a B200): the n_split
+ * in 1 .. 8 whose CTA waves times longest part is smallest (the smaller on a
+ * tie), and the workspace bytes it needs (0 for 1).  Host only; no CUDA call. */
+int kvq_prefill_split(const kvq_pool_desc *desc, int pos0, int n_tok, int n_sms, int *n_split,
+                      uint64_t *workspace_bytes);
 
 /* attn_combine: for each (sequence, query head), merge the partials of its
  * units with the log-sum-exp rule (M = max m_j, L = sum l_j 2^(m_j - M),

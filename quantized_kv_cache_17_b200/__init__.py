@@ -39,7 +39,7 @@ EXPORTS = ["kvq_version", "kvq_pool_bytes", "kvq_pool_layout", "q_rotate", "kv_a
            "paged_decode_attn_fp8_combined", "paged_decode_attn_nvfp4_combined",
            "paged_decode_attn_q4_0_noalloc", "paged_decode_attn_cudacore", "attn_combine",
            "paged_decode_step_int8", "paged_decode_step_q4_0", "paged_decode_step_k8v4",
-           "paged_decode_step_fp8", "paged_decode_step_nvfp4", "paged_prefill_attn",
+           "paged_decode_step_fp8", "paged_decode_step_nvfp4", "paged_prefill_attn", "kvq_prefill_split",
            "kvq_resident_state_bytes", "kvq_resident_init", "kvq_resident_map", "kvq_resident_load",
            "kvq_resident_query", "kvq_resident_stats"]
 _FMT_NAMES = ("int8", "q4_0", "k8v4", "fp8", "nvfp4")
@@ -99,7 +99,10 @@ def lib():
             getattr(L, "paged_decode_step_" + f).argtypes = [ctypes.POINTER(Pool), I32, P, P, P, P, I32, P,
                                                              ctypes.POINTER(PlanInfo), P, ctypes.c_uint64, P, P, P, P]
         L.attn_combine.argtypes = [P, P, ctypes.POINTER(PlanInfo), I32, P, P, P]
-        L.paged_prefill_attn.argtypes = [ctypes.POINTER(Pool), I32, P, I32, I32, I32, P, I32, I32, P, P, P, P]
+        L.paged_prefill_attn.argtypes = [ctypes.POINTER(Pool), I32, P, I32, I32, I32, P, I32, I32, I32, P,
+                                         ctypes.c_uint64, P, P, P, P]
+        L.kvq_prefill_split.argtypes = [ctypes.POINTER(PoolDesc), I32, I32, I32, ctypes.POINTER(ctypes.c_int),
+                                        ctypes.POINTER(ctypes.c_uint64)]
         L.kvq_resident_init.argtypes = [P, ctypes.c_uint64, ctypes.POINTER(Pool), ctypes.POINTER(Pool)]
         L.kvq_resident_map.argtypes = [P, I32, P, I32, I32, P, P, P, I32, ctypes.POINTER(ctypes.c_int)]
         L.kvq_resident_load.argtypes = [P, I32, P, I32, P]
@@ -296,16 +299,35 @@ def paged_decode_attn_nvfp4(pool, layer, q, page_table, plan_dev, info, workspac
     paged_decode_attn(pool, layer, q, page_table, plan_dev, info, workspace, status, stream)
 
 
+def prefill_split(desc: PoolDesc, pos0: int, n_tok: int, n_sms: int = 0):
+    """(n_split, workspace bytes) the library suggests for a prefill chunk."""
+    ns, wb = ctypes.c_int(), ctypes.c_uint64()
+    _check(lib().kvq_prefill_split(ctypes.byref(desc), pos0, n_tok, n_sms, ctypes.byref(ns), ctypes.byref(wb)),
+           "kvq_prefill_split")
+    return ns.value, wb.value
+
+
 def paged_prefill_attn(pool: KVPool, layer: int, q, seq: int, pos0: int, page_table, out_bf16, out_f32=None,
-                       status=None, stream=None):
+                       status=None, stream=None, n_split=None, workspace=None):
     """Chunked-prefill attention: q [n_tok, n_q_heads, 256] (prepared as for
     the decode) of sequence seq at positions pos0 .. pos0 + n_tok - 1, whose
-    keys are already in the pool, attends causally over the sequence's cache."""
+    keys are already in the pool, attends causally over the sequence's cache.
+    n_split None takes kvq_prefill_split's choice; a workspace the split needs
+    and the caller does not pass is allocated here (as a torch tensor)."""
     cp = pool.c_pool()
     n_tok = q.shape[0]
+    if n_split is None:
+        n_split, wb = prefill_split(pool.desc, pos0, n_tok)
+    else:
+        wb = n_split * pool.desc.n_q_heads * n_tok * 260 * 4 if n_split > 1 else 0
+    if n_split > 1 and workspace is None:
+        import torch
+        workspace = torch.empty(wb // 4, dtype=torch.float32, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().paged_prefill_attn(ctypes.byref(cp), layer, _ptr(q), seq, pos0, n_tok, _ptr(page_table),
-                                    page_table.shape[1], page_table.shape[0], _ptr(out_bf16), _ptr(out_f32),
-                                    _ptr(status), _stream(stream)), "paged_prefill_attn")
+                                    page_table.shape[1], page_table.shape[0], n_split, _ptr(workspace), ws_bytes,
+                                    _ptr(out_bf16), _ptr(out_f32), _ptr(status), _stream(stream)),
+           "paged_prefill_attn")
 
 
 def attn_combine(workspace, plan_dev, info: PlanInfo, inverse_fwht: bool, out_bf16, out_f32=None, stream=None):

@@ -322,9 +322,39 @@ KVQ_STEP(paged_decode_step_fp8, KVQ_FP8)
 KVQ_STEP(paged_decode_step_nvfp4, KVQ_NVFP4)
 #undef KVQ_STEP
 
+int kvq_prefill_split(const kvq_pool_desc *desc, int pos0, int n_tok, int n_sms, int *n_split,
+                      uint64_t *workspace_bytes) {
+    uint64_t pb = 0;
+    if (!desc || !n_split || !workspace_bytes) return KVQ_EINVAL;
+    const int rc = kvq_pool_bytes(desc, &pb);
+    if (rc) return rc;
+    if (n_tok <= 0 || pos0 < 0 || (int64_t)pos0 + n_tok > INT32_MAX || n_sms < 0) return KVQ_EINVAL;
+    const int sms = n_sms ? n_sms : 148;
+    const int G = desc->n_q_heads / desc->n_kv_heads;
+    const int64_t n_rows = (int64_t)n_tok * G;
+    const int64_t ctas = (n_rows + 63) / 64 * desc->n_kv_heads;    // CTAs of one part (64 rows each)
+    const int64_t t_end = (int64_t)pos0 + n_tok;
+    // cost of a choice: waves of CTAs times the longest part
+    int best = 1;
+    int64_t best_cost = (ctas + sms - 1) / sms * t_end;
+    for (int s = 2; s <= PF_MAX_SPLIT; ++s) {
+        const int st = prefill_split_tokens(pos0, n_tok, s);
+        if (!st) break;
+        const int64_t longest = std::max<int64_t>(st, t_end - (int64_t)(s - 1) * st);
+        const int64_t cost = (ctas * s + sms - 1) / sms * longest;
+        if (cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    *n_split = best;
+    *workspace_bytes = best > 1 ? (uint64_t)best * desc->n_kv_heads * n_rows * PF_WS_STRIDE * sizeof(float) : 0;
+    return KVQ_OK;
+}
+
 int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq, int pos0, int n_tok,
-                       const int32_t *page_table, int max_pages, int n_seq, uint16_t *out_bf16, float *out_f32,
-                       int32_t *status, void *stream) {
+                       const int32_t *page_table, int max_pages, int n_seq, int n_split, float *workspace,
+                       uint64_t workspace_bytes, uint16_t *out_bf16, float *out_f32, int32_t *status, void *stream) {
     PoolGeom geo;
     const int rc = check_pool(pool, layer, &geo);
     if (rc) return rc;
@@ -332,10 +362,20 @@ int paged_prefill_attn(const kvq_pool *pool, int layer, const float *q, int seq,
         return KVQ_EINVAL;
     if ((int64_t)max_pages * PAGE > INT32_MAX || (int64_t)pos0 + n_tok > (int64_t)max_pages * PAGE) return KVQ_EINVAL;
     if ((int64_t)n_tok * pool->desc.n_q_heads > ((int64_t)1 << 28)) return KVQ_EINVAL;
+    if (n_split < 1 || n_split > PF_MAX_SPLIT) return KVQ_EINVAL;
+    const int split_tokens = prefill_split_tokens(pos0, n_tok, n_split);
+    if (n_split > 1) {
+        if (!split_tokens || !workspace) return KVQ_EINVAL;
+        const uint64_t need = (uint64_t)n_split * pool->desc.n_kv_heads * ((uint64_t)n_tok * pool->desc.n_q_heads /
+                                                                            pool->desc.n_kv_heads) *
+                              PF_WS_STRIDE * sizeof(float);
+        if (workspace_bytes < need) return KVQ_ESIZE;
+        if (!aligned16(workspace)) return KVQ_EALIGN;
+    }
     if (!aligned16(q) || !aligned16(out_bf16) || (out_f32 && !aligned16(out_f32))) return KVQ_EALIGN;
     return cuda_rc(launch_prefill(pool->desc.fmt, static_cast<const uint8_t *>(pool->base), geo, layer, q, seq, pos0,
-                                  n_tok, page_table, max_pages, pool->desc.n_q_heads,
-                                  host_rotated_v(pool->desc.fmt) ? 1 : 0, out_bf16, out_f32, status,
+                                  n_tok, page_table, max_pages, pool->desc.n_q_heads, n_split, split_tokens,
+                                  workspace, host_rotated_v(pool->desc.fmt) ? 1 : 0, out_bf16, out_f32, status,
                                   static_cast<cudaStream_t>(stream)));
 }
 

@@ -1737,6 +1737,8 @@ __global__ void __launch_bounds__(TcCfg<FMT>::NTHREADS, 1) decode_tc_kernel(cons
 struct PrefillArgs {
     DecodeArgs d;            // pool, geometry, layer, page table, status (the copy loop's view)
     int seq, pos0, n_tok, n_rows;
+    int n_split, split_tokens;   // key range cut at multiples of split_tokens (blockIdx.z = part)
+    float *ws;                   // n_split > 1: partials [part][kv head][row][PF_WS_STRIDE]
 };
 
 template <int FMT> struct PfCfg {
@@ -1780,8 +1782,17 @@ __global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(con
     // keys 0 .. pos0 + (last token of the CTA's rows)
     const int i_last = min(P.n_tok - 1, (r0 + C::ROWS - 1) / G);
     const int t_end = P.pos0 + i_last + 1;
-    const int n_steps = (t_end + STEP_TOKENS - 1) / STEP_TOKENS;
-    const int n_items = (t_end + C::TPI * TILE - 1) / (C::TPI * TILE);
+    // this CTA's part of the key range: [t0, t1).  Every cut lies at or below
+    // pos0, so every row sees the first key of its part.
+    const int part = blockIdx.z;
+    const int t0 = part * P.split_tokens;
+    const int t1 = part == P.n_split - 1 ? t_end : min(t_end, t0 + P.split_tokens);
+    if (t1 <= t0) {                            // excluded by the host; kept as a guard
+        if (threadIdx.x == 0) status_or(A.status, KVQ_STATUS_BAD_PLAN);
+        return;
+    }
+    const int n_steps = (t1 - t0 + STEP_TOKENS - 1) / STEP_TOKENS;
+    const int n_items = (t1 - t0 + C::TPI * TILE - 1) / (C::TPI * TILE);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NS; ++i) {
@@ -1794,7 +1805,7 @@ __global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(con
     __syncthreads();
 
     if (warp == C::COPY_WARP) {
-        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, P.seq, kvh, 0, n_steps, lane);
+        copy_loop<C::NS, C::STAGE_BYTES, L::BYTES>(A, smem, full, empty, stage_ok, P.seq, kvh, t0, n_steps, lane);
         return;
     }
     if (warp == C::SCALE_WARP) {
@@ -1831,10 +1842,10 @@ __global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(con
             if (lane == 0) status_or(A.status, KVQ_STATUS_TIMEOUT);
             break;
         }
-        const int tok = it * C::TPI * TILE;
+        const int tok = t0 + it * C::TPI * TILE;
         int v[C::TPI];
 #pragma unroll
-        for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t_end - tok - j * TILE));
+        for (int j = 0; j < C::TPI; ++j) v[j] = max(0, min(TILE, t1 - tok - j * TILE));
         const uint8_t *tp = smem + si * C::STAGE_BYTES + within * C::TPI * L::BYTES;
         const bool ok = stage_ok[si] != 0;
         if (ok) {
@@ -1862,8 +1873,28 @@ __global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(con
     lr += __shfl_xor_sync(0xffffffffu, lr, 1);
     lr += __shfl_xor_sync(0xffffffffu, lr, 2);            // row g's sum on lanes 4g .. 4g+3
     const int t = lane & 3;
-    const float l0 = __shfl_sync(0xffffffffu, lr, 8 * t), l1 = __shfl_sync(0xffffffffu, lr, 8 * t + 4);
     float *b = reinterpret_cast<float *>(smem) + warp * 8 * T::OSTRIDE;
+    if (P.ws) {
+        // a part of the key range: o unnormalised with its (m, l), merged later
+        pv.store_scaled(b, 1.f, 1.f, lane);
+        __syncwarp();
+        float *wsp = P.ws + ((size_t)part * A.geo.n_kv_heads + kvh) * (size_t)P.n_rows * PF_WS_STRIDE;
+        const int rh = r0 + 8 * warp + (lane >> 2);
+        if ((lane & 3) == 0 && rh < P.n_rows) {
+            wsp[(size_t)rh * PF_WS_STRIDE + D] = qk.m_run;
+            wsp[(size_t)rh * PF_WS_STRIDE + D + 1] = lr;
+        }
+        for (int h = 0; h < 8; ++h) {
+            const int rr = r0 + 8 * warp + h;
+            if (rr >= P.n_rows) break;
+            const float *src = b + h * T::OSTRIDE + lane * 8;
+            float4 *dst = reinterpret_cast<float4 *>(wsp + (size_t)rr * PF_WS_STRIDE + lane * 8);
+            dst[0] = make_float4(src[0], src[1], src[2], src[3]);
+            dst[1] = make_float4(src[4], src[5], src[6], src[7]);
+        }
+        return;
+    }
+    const float l0 = __shfl_sync(0xffffffffu, lr, 8 * t), l1 = __shfl_sync(0xffffffffu, lr, 8 * t + 4);
     pv.store_scaled(b, l0 > 0.f ? 1.f / l0 : 0.f, l1 > 0.f ? 1.f / l1 : 0.f, lane);
     __syncwarp();
     for (int h = 0; h < 8; ++h) {
@@ -1875,6 +1906,38 @@ __global__ void __launch_bounds__(PfCfg<FMT>::NTHREADS, 1) prefill_tc_kernel(con
         const int ti = rr / G, hh = rr % G;
         finish_row(x, lane, A.inverse_fwht, (int64_t)ti * A.n_q_heads + (int64_t)kvh * G + hh, A.out_bf16, A.out_f32);
     }
+}
+
+// Merge of the key-range parts of a split prefill: one warp per (KV head, row),
+// the log-sum-exp rule over the parts, then 1/L and the output rotation.
+__global__ void __launch_bounds__(256) prefill_merge_kernel(const float *__restrict__ ws, int n_split, int n_kv,
+                                                            int n_rows, int G, int n_q_heads, int inverse_fwht,
+                                                            uint16_t *out_bf16, float *out_f32) {
+    grid_dependency_wait();
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= n_kv * n_rows) return;            // warp-uniform
+    const int kvh = w / n_rows, r = w - kvh * n_rows;
+    const size_t part_stride = (size_t)n_kv * n_rows * PF_WS_STRIDE;
+    const float *row = ws + ((size_t)kvh * n_rows + r) * PF_WS_STRIDE;
+    float M = -INFINITY;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, row[s * part_stride + D]);
+    float L = 0.f, x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < n_split; ++s) {
+        const float *p = row + s * part_stride;
+        const float m = p[D];
+        if (m == -INFINITY) continue;
+        const float f = exp2f(m - M);
+        L += f * p[D + 1];
+        const float4 a = reinterpret_cast<const float4 *>(p + lane * 8)[0];
+        const float4 b = reinterpret_cast<const float4 *>(p + lane * 8)[1];
+        x[0] += f * a.x; x[1] += f * a.y; x[2] += f * a.z; x[3] += f * a.w;
+        x[4] += f * b.x; x[5] += f * b.y; x[6] += f * b.z; x[7] += f * b.w;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] *= inv;
+    const int ti = r / G, hh = r - ti * G;
+    finish_row(x, lane, inverse_fwht, (int64_t)ti * n_q_heads + (int64_t)kvh * G + hh, out_bf16, out_f32);
 }
 
 // ---------------------------------------------------------------------------
@@ -2088,13 +2151,20 @@ cudaError_t launch_prefill_fmt(const PrefillArgs &p, cudaStream_t s) {
             configured[dev] = true;
         }
     }
-    const dim3 grid((unsigned)((p.n_rows + C::ROWS - 1) / C::ROWS), (unsigned)p.d.geo.n_kv_heads);
-    return launch_ex(prefill_tc_kernel<FMT>, grid, dim3(C::NTHREADS), C::TOTAL, s, false, p);
+    const dim3 grid((unsigned)((p.n_rows + C::ROWS - 1) / C::ROWS), (unsigned)p.d.geo.n_kv_heads,
+                    (unsigned)p.n_split);
+    cudaError_t e = launch_ex(prefill_tc_kernel<FMT>, grid, dim3(C::NTHREADS), C::TOTAL, s, false, p);
+    if (e != cudaSuccess || !p.ws) return e;
+    const int warps = p.d.geo.n_kv_heads * p.n_rows;
+    return launch_ex(prefill_merge_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, false,
+                     (const float *)p.ws, p.n_split, p.d.geo.n_kv_heads, p.n_rows, p.d.G, p.d.n_q_heads,
+                     p.d.inverse_fwht, p.d.out_bf16, p.d.out_f32);
 }
 
 cudaError_t launch_prefill(int fmt, const uint8_t *pool, const PoolGeom &geo, int layer, const float *q, int seq,
                            int pos0, int n_tok, const int32_t *page_table, int max_pages, int n_q_heads,
-                           int inverse_fwht, uint16_t *out_bf16, float *out_f32, int32_t *status, cudaStream_t s) {
+                           int n_split, int split_tokens, float *ws, int inverse_fwht, uint16_t *out_bf16,
+                           float *out_f32, int32_t *status, cudaStream_t s) {
     const int G = n_q_heads / geo.n_kv_heads;
     PrefillArgs p{};
     p.d = DecodeArgs{pool, geo, layer, q, page_table, max_pages, nullptr, n_q_heads, G, nullptr,
@@ -2103,6 +2173,9 @@ cudaError_t launch_prefill(int fmt, const uint8_t *pool, const PoolGeom &geo, in
     p.pos0 = pos0;
     p.n_tok = n_tok;
     p.n_rows = n_tok * G;
+    p.n_split = n_split;
+    p.split_tokens = split_tokens;
+    p.ws = n_split > 1 ? ws : nullptr;
     switch (fmt) {
     case KVQ_INT8: return launch_prefill_fmt<KVQ_INT8>(p, s);
     case KVQ_Q4_0: return launch_prefill_fmt<KVQ_Q4_0>(p, s);

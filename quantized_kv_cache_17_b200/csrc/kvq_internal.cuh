@@ -345,7 +345,26 @@ cudaError_t launch_append_rotate(int fmt, uint8_t *pool, const PoolGeom &geo, in
                                  float *q_rot, int64_t n_vec, cudaStream_t s);
 cudaError_t launch_prefill(int fmt, const uint8_t *pool, const PoolGeom &geo, int layer, const float *q, int seq,
                            int pos0, int n_tok, const int32_t *page_table, int max_pages, int n_q_heads,
-                           int inverse_fwht, uint16_t *out_bf16, float *out_f32, int32_t *status, cudaStream_t s);
+                           int n_split, int split_tokens, float *ws, int inverse_fwht, uint16_t *out_bf16,
+                           float *out_f32, int32_t *status, cudaStream_t s);
+
+// Split prefill: floats per (part, KV head, row) partial: o[256], m, l, padding.
+constexpr int PF_WS_STRIDE = 260;
+constexpr int PF_MAX_SPLIT = 8;
+
+// Length of every part but the last when the key range [0, pos0 + n_tok) of a
+// prefill is cut into n_split parts: a multiple of 64 tokens (the copy step),
+// about an equal share, and small enough that every cut lies at or below pos0
+// (so each row of the chunk sees the first key of every part).  0 when no such
+// cut exists.
+inline int prefill_split_tokens(int pos0, int n_tok, int n_split) {
+    if (n_split <= 1) return 0;
+    const int64_t t_end = (int64_t)pos0 + n_tok;
+    const int64_t share = (t_end + 64LL * n_split - 1) / (64LL * n_split) * 64;
+    const int64_t cap = ((int64_t)(pos0 & ~63) / (n_split - 1)) & ~63LL;
+    const int64_t st = share < cap ? share : cap;
+    return st >= 64 ? (int)st : 0;
+}
 cudaError_t launch_decode(int fmt, bool tensor_cores, const uint8_t *pool, const PoolGeom &geo, int layer,
                           const float *q, const int32_t *page_table, int max_pages, const int32_t *plan,
                           const kvq_plan_info &info, float *ws, int32_t *status, int inverse_fwht,

@@ -35,7 +35,7 @@ def _workload(fmt, Hq, Hkv, T, name, order="permuted", outlier="mul20", q_post=1
                                q_outliers=q_outliers)
 
 
-def _prefill(w, n_tok, split=None):
+def _prefill(w, n_tok, split=None, n_split=None):
     """Pool with the sequence's tokens [0, T - 1); the chunk [T - n_tok, T) appended
     in one kv_append call; then the prefill of the chunk (in calls of `split`
     tokens when given).  Returns (dw, pos0, out_f32 [n_tok, Hq, 256], out_bf16)."""
@@ -57,7 +57,7 @@ def _prefill(w, n_tok, split=None):
     for c0 in range(0, n_tok, step):
         c1 = min(n_tok, c0 + step)
         kvq.paged_prefill_attn(dw.pool, 0, qp[c0:c1].contiguous(), 0, pos0 + c0, dw.page_table, out_bf[c0:c1],
-                               out_f[c0:c1], status=status)
+                               out_f[c0:c1], status=status, n_split=n_split)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return dw, pos0, out_f.cpu().numpy(), out_bf.cpu()
@@ -110,14 +110,38 @@ def test_prefill_32k_chunks(n_tok):
 
 @pytest.mark.parametrize("fmt", ["q4_0", "k8v4"])
 def test_prefill_in_smaller_chunks_is_bit_identical(fmt):
-    """Each row's result depends only on its own keys: splitting the chunk
-    into calls of 16 and 40 tokens gives the same bits as one call."""
+    """Without a key-range split each row's result depends only on its own
+    keys: cutting the chunk into calls of 16 and 40 tokens gives the same bits
+    as one call."""
     w = _workload(fmt, 12, 2, 900, f"prefill_split_{fmt}")
-    _, _, one, one_bf = _prefill(w, 80)
+    _, _, one, one_bf = _prefill(w, 80, n_split=1)
     for split in (16, 40):
-        _, _, parts, parts_bf = _prefill(w, 80, split=split)
+        _, _, parts, parts_bf = _prefill(w, 80, split=split, n_split=1)
         assert np.array_equal(parts.view(np.uint32), one.view(np.uint32))
         assert torch.equal(parts_bf.view(torch.int16), one_bf.view(torch.int16))
+
+
+@pytest.mark.parametrize("n_split", [1, 2, 3, 8])
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_prefill_key_split_matches_oracle(fmt, n_split):
+    """The key range cut into n_split parts (cuts at multiples of 64 at or below
+    pos0), partials merged by the second kernel: every row against the oracle."""
+    w = _workload(fmt, 12, 2, 1400, f"prefill_ks_{fmt}_{n_split}")
+    dw, pos0, out_f, out_bf = _prefill(w, 37, n_split=n_split)
+    _check_rows(w, dw, pos0, out_f, out_bf, list(range(37)), list(range(w.n_kv_heads)))
+
+
+def test_prefill_default_split_at_32k():
+    """The split kvq_prefill_split picks for a 512-token chunk at 32,768 (the
+    bench's case) against the unsplit kernel and the oracle on sampled rows."""
+    w = _workload("q4_0", 24, 4, 32768, "prefill32k_auto", order="contiguous", outlier="student_t",
+                  q_post=1 / 16, q_outliers=False, n_out=8)
+    n_split, wb = kvq.prefill_split(kvq.make_desc(1, 4, 24, 128, "q4_0"), 32768 - 512, 512)
+    assert n_split > 1 and wb > 0
+    dw, pos0, out_f, out_bf = _prefill(w, 512)
+    _, _, one_f, _ = _prefill(w, 512, n_split=1)
+    gc.assert_close(out_f.reshape(-1, 256), one_f.reshape(-1, 256), "split vs unsplit")
+    _check_rows(w, dw, pos0, out_f, out_bf, [0, 255, 511], [0, 3])
 
 
 def test_prefill_rejects_bad_arguments():
@@ -130,3 +154,11 @@ def test_prefill_rejects_bad_arguments():
             kvq.paged_prefill_attn(dw.pool, 0, q, 0, pos0, dw.page_table, out)
     with pytest.raises(kvq.KVQError, match="KVQ_EINVAL"):
         kvq.paged_prefill_attn(dw.pool, 0, q, 1, 0, dw.page_table, out)           # seq out of range
+    for bad in (0, 9):
+        with pytest.raises(kvq.KVQError, match="KVQ_EINVAL"):
+            kvq.paged_prefill_attn(dw.pool, 0, q, 0, 200, dw.page_table, out, n_split=bad)
+    with pytest.raises(kvq.KVQError, match="KVQ_EINVAL"):                           # no cut at or below pos0
+        kvq.paged_prefill_attn(dw.pool, 0, q, 0, 100, dw.page_table, out, n_split=3)
+    small = torch.empty(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(kvq.KVQError, match="KVQ_ESIZE"):
+        kvq.paged_prefill_attn(dw.pool, 0, q, 0, 200, dw.page_table, out, n_split=2, workspace=small)

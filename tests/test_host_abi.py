@@ -151,3 +151,41 @@ def test_validation_errors_without_a_gpu():
     assert L.paged_decode_attn_nvfp4(*args, info.workspace_bytes, None, None) == -1
     bad = kvq.make_desc(1, 4, 24, 8, 5)                                                     # no such format
     assert L.kvq_pool_bytes(ctypes.byref(bad), ctypes.byref(ctypes.c_uint64())) == -1
+
+
+@pytest.mark.parametrize("pos0,n_tok", [(32256, 512), (0, 512), (100, 512), (64, 100), (1000, 1), (261632, 512),
+                                        (5000, 3000), (63, 1), (64, 1)])
+def test_prefill_split_choice(pos0, n_tok):
+    """kvq_prefill_split: a valid cut (multiples of 64, all at or below pos0),
+    the workspace it needs, and never more waves x longest part than no split."""
+    d = kvq.make_desc(1, 4, 24, 1100, "q4_0")
+    ns, wb = kvq.prefill_split(d, pos0, n_tok)
+    assert 1 <= ns <= 8
+    assert wb == (ns * 4 * n_tok * 6 * 260 * 4 if ns > 1 else 0)
+    if ns > 1:
+        t_end = pos0 + n_tok
+        share = -(-t_end // (64 * ns)) * 64
+        st = min(share, ((pos0 // 64 * 64) // (ns - 1)) // 64 * 64)
+        assert st >= 64 and (ns - 1) * st <= pos0 and st % 64 == 0
+        ctas = -(-n_tok * 6 // 64) * 4
+        assert -(-ctas * ns // 148) * max(st, t_end - (ns - 1) * st) < -(-ctas // 148) * t_end
+    if pos0 < 64:
+        assert ns == 1
+
+
+def test_prefill_validation_without_a_gpu():
+    L = kvq.lib()
+    d = kvq.make_desc(1, 2, 12, 8, "q4_0")
+    pool = kvq.Pool(0x10000, d)
+    args = (ctypes.byref(pool), 0, 0x1000, 0, 256, 4, 0x2000, 8, 1)
+    tail = (0x3000, 0x4000, None, None)
+    assert L.paged_prefill_attn(*args, 0, None, 0, *tail) == -1            # n_split 0
+    assert L.paged_prefill_attn(*args, 9, None, 0, *tail) == -1            # above 8
+    assert L.paged_prefill_attn(*args, 2, None, 0, *tail) == -1            # split without a workspace
+    assert L.paged_prefill_attn(*args, 2, 0x5000, 100, *tail) == -5        # workspace too small
+    assert L.paged_prefill_attn(*args, 2, 0x5008, 1 << 30, *tail) == -3    # unaligned workspace
+    args_low = (ctypes.byref(pool), 0, 0x1000, 0, 100, 4, 0x2000, 8, 1)
+    assert L.paged_prefill_attn(*args_low, 3, 0x5000, 1 << 30, *tail) == -1   # no cut at or below pos0
+    ns, wb = ctypes.c_int(), ctypes.c_uint64()
+    assert L.kvq_prefill_split(ctypes.byref(d), -1, 4, 0, ctypes.byref(ns), ctypes.byref(wb)) == -1
+    assert L.kvq_prefill_split(ctypes.byref(d), 0, 0, 0, ctypes.byref(ns), ctypes.byref(wb)) == -1
