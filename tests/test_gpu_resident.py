@@ -106,3 +106,39 @@ def test_resident_load_rejects_device_memory_as_host_pool():
     _, loads = rc.map(0, np.array([[0]], np.int32), [10])
     with pytest.raises(kvq.KVQError, match="EINVAL"):
         rc.load(0, loads)
+
+
+@pytest.mark.parametrize("fmt", ["q4_0", "k8v4"])
+def test_resident_prefill_is_bit_identical(fmt):
+    """A prompt chunk appended and attended through the page cache gives the same
+    bits as through the full device pool, unsplit and with a key-range split."""
+    base = dataclasses.replace(kvq_inputs.workload("ragged4_q4_0"), fmt=fmt)
+    w = kvq_inputs.scaled(base, [1800, 900], n_layers=2)
+    dw = kdev.build_pool(w)
+    D = dw.pool
+    H = kvq.KVPool.allocate(D.desc, "pinned")
+    H.buf.copy_(D.buf)
+    C = kvq.KVPool.allocate(kvq.make_desc(1, w.n_kv_heads, w.n_q_heads, 12, fmt))
+    rc = kvq.ResidentCache(H, C)
+    n_tok = 40
+    for layer in range(w.n_layers):
+        T = w.seq_lens[0]
+        pos0 = T - 1 - n_tok            # the chunk ends one token before the pool's fill
+        cpt, loads = rc.map(layer, dw.page_table_host, [T, w.seq_lens[1]])
+        rc.load(layer, loads)
+        cpt_d = torch.from_numpy(cpt).cuda()
+        qt = kdev.DeviceTable(w.q_table(layer), "cuda")
+        q = kdev.gen_rows_device(w.q_key(layer, 0), qt, 0, n_tok)
+        qp = kvq.q_rotate(q) if kvq.rotated_q(fmt) else q
+        for n_split in (1, 3):
+            outs = []
+            for pool, lay, pt in ((D, layer, dw.page_table), (C, 0, cpt_d)):
+                o_bf = torch.empty((n_tok, w.n_q_heads, 256), dtype=torch.bfloat16, device="cuda")
+                o_f = torch.empty((n_tok, w.n_q_heads, 256), dtype=torch.float32, device="cuda")
+                st = torch.zeros(1, dtype=torch.int32, device="cuda")
+                kvq.paged_prefill_attn(pool, lay, qp, 0, pos0, pt, o_bf, o_f, status=st, n_split=n_split)
+                torch.cuda.synchronize()
+                assert int(st.item()) == 0
+                outs.append((o_f, o_bf))
+            assert torch.equal(outs[0][0].view(torch.int32), outs[1][0].view(torch.int32)), (fmt, layer, n_split)
+            assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
