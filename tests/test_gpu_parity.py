@@ -161,6 +161,30 @@ def test_decode_matches_oracle(case, fmt, impl):
         gc.assert_bf16_consistent(out_f, out_bf, ref_all)
 
 
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 7])
+@pytest.mark.parametrize("fmt", ["int8", "q4_0", "k8v4", "fp8", "nvfp4"])
+def test_decode_every_group_size(fmt, G):
+    """Group sizes the shipped configurations do not use (1 = one query head
+    per KV head, up to 7), in the split and fused forms and as the one-launch
+    step, against the oracle."""
+    w = small(fmt, 2 * G, 2, [700, 1, 257], outlier="student_t", q_post=1 / 16, q_outliers=False, n_out=8,
+              name=f"groups_{fmt}_{G}")
+    dw = kdev.build_pool(w, extra_slots=1)
+    q, k, v, pos = kdev.step_inputs(w, [0])
+    kvq.kv_append(dw.pool, 0, k[0], v[0], pos, dw.page_table)
+    refs = {(b, g): gc.oracle_group(dw, 0, b, g) for b in range(w.batch) for g in range(w.n_kv_heads)}
+    for mode, n_ctas in (("split", 0), ("fused", 7)):
+        out_f, out_bf, status, _, _ = gc.decode_step(dw, 0, q[0], n_ctas=n_ctas, mode=mode)
+        assert status == 0
+        for (b, g), ref in refs.items():
+            gc.assert_close(out_f[b, g * G:(g + 1) * G], ref, f"G={G}/{fmt}/{mode} b={b} g={g}")
+    # the step appends the same token again (same bytes) and must give the same answer
+    out_s, _, status, _, _ = gc.decode_step(dw, 0, q[0], mode="step", k_new=k[0], v_new=v[0])
+    assert status == 0
+    for (b, g), ref in refs.items():
+        gc.assert_close(out_s[b, g * G:(g + 1) * G], ref, f"G={G}/{fmt}/step b={b} g={g}")
+
+
 def test_decode_single_token_context():
     """T = 1: the output is that token's dequantised value, un-rotated."""
     w = small("q4_0", 6, 1, [1])

@@ -131,6 +131,16 @@ def test_prefill_key_split_matches_oracle(fmt, n_split):
     _check_rows(w, dw, pos0, out_f, out_bf, list(range(37)), list(range(w.n_kv_heads)))
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (8, 1), (6, 2), (14, 2)])
+def test_prefill_group_sizes(Hq, Hkv):
+    """Group sizes 1, 8, 3 and 7: the rows r = i G + h of a CTA span token
+    boundaries differently for each."""
+    w = _workload("q4_0", Hq, Hkv, 900, f"prefill_g_{Hq}_{Hkv}")
+    for n_split in (1, 2):
+        dw, pos0, out_f, out_bf = _prefill(w, 23, n_split=n_split)
+        _check_rows(w, dw, pos0, out_f, out_bf, list(range(23)), list(range(w.n_kv_heads)))
+
+
 def test_prefill_default_split_at_32k():
     """The split kvq_prefill_split picks for a 512-token chunk at 32,768 (the
     bench's case) against the unsplit kernel and the oracle on sampled rows."""
