@@ -226,19 +226,27 @@ __device__ __forceinline__ void convert_stage_scales(const uint8_t *stage, float
         *reinterpret_cast<float2 *>(sf + tile * TcCfg<FMT>::SF_TILE + pair * TcCfg<FMT>::KSTRIDE) = d;
         return;
     } else if constexpr (L::KP == PART_F4) {
-        constexpr int KSTRIDE = TcCfg<FMT>::KSTRIDE;
+        // lane: tile lane / 4, tokens 2 (lane % 4) and 2 (lane % 4) + 1; word 16 r + b of
+        // the tile's row = the scale of token r, block b as the fp16 pair (s, s)
+        const int tile = lane >> 2, pair = lane & 3;
+        uint32_t *dst = reinterpret_cast<uint32_t *>(sf) + tile * TcCfg<FMT>::SF_TILE + 32 * pair;
 #pragma unroll
-        for (int c = lane; c < 8 * 8; c += 32) {            // 8 chunks of 16 bytes per tile
-            const int tile = c >> 3, pair = (c >> 1) & 3, half = c & 1;
+        for (int half = 0; half < 2; ++half) {
             const uint4 h = lds128(stage + tile * L::BYTES + L::KS + pair * 32 + half * 16);
-            float *dst = sf + tile * 4 * KSTRIDE + pair * KSTRIDE + half * 16;
+            uint32_t ev[8], od[8];                          // blocks 8 half .. 8 half + 7
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t w = u4_at(h, i);
-                const float2 a = __half22float2(u32_as_h2(e4m3x2_to_h2(w)));
-                const float2 b = __half22float2(u32_as_h2(e4m3x2_to_h2(w >> 16)));
-                *reinterpret_cast<float4 *>(dst + 4 * i) = make_float4(a.x, a.y, b.x, b.y);
+                const uint32_t w = u4_at(h, i);             // bytes: (b, even), (b, odd), (b + 1, even), (b + 1, odd)
+                const uint32_t x = e4m3x2_to_h2(w), y = e4m3x2_to_h2(w >> 16);
+                ev[2 * i] = __byte_perm(x, 0, 0x1010);
+                od[2 * i] = __byte_perm(x, 0, 0x3232);
+                ev[2 * i + 1] = __byte_perm(y, 0, 0x1010);
+                od[2 * i + 1] = __byte_perm(y, 0, 0x3232);
             }
+            sts128(dst + 8 * half, make_uint4(ev[0], ev[1], ev[2], ev[3]));
+            sts128(dst + 8 * half + 4, make_uint4(ev[4], ev[5], ev[6], ev[7]));
+            sts128(dst + 16 + 8 * half, make_uint4(od[0], od[1], od[2], od[3]));
+            sts128(dst + 16 + 8 * half + 4, make_uint4(od[4], od[5], od[6], od[7]));
         }
         return;
     }
@@ -442,31 +450,51 @@ template <int FMT> struct QkWarp {
             s[3] = ((c[0][1] + c[0][3]) + (c[1][1] + c[1][3])) * dB.y;
             return;
         } else if constexpr (L::KP == PART_F4) {
-            // E2M1 keys: one k-step per 16-value block, each with its own scale
-#pragma unroll
-            for (int i = 0; i < 4; ++i) s[i] = 0.f;
+            // E2M1 keys: a value times its E4M3 scale has at most 6 significant
+            // bits and lies in [2^-10, 2688], so the fp16 product is the exact key
+            // and the 16 k-steps of a tile accumulate in one product (two chains)
+            const int g = lane >> 2;
+            const uint32_t *sfA = reinterpret_cast<const uint32_t *>(fA) + 16 * g;     // token g's 16 scale pairs
+            const uint32_t *sfB = reinterpret_cast<const uint32_t *>(fB) + 16 * g;
+            float a[2][4], c[2][4];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const uint4 kA = lds128(tA + L::KC + hf * 512 + lane * 16);
                 const uint4 kB = lds128(tB + L::KC + hf * 512 + lane * 16);
+                const uint4 sA0 = lds128(sfA + 8 * hf), sA1 = lds128(sfA + 8 * hf + 4);
+                const uint4 sB0 = lds128(sfB + 8 * hf), sB1 = lds128(sfB + 8 * hf + 4);
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb) {
                     const int b = 4 * hf + bb;              // 32 dims: k-steps 2b, 2b + 1
                     const uint32_t wA = u4_at(kA, bb), wB = u4_at(kB, bb);
-                    float a0[4], a1[4], c0[4], c1[4];
+                    const uint32_t xA0 = u4_at(bb < 2 ? sA0 : sA1, (2 * bb) & 3), xA1 = u4_at(bb < 2 ? sA0 : sA1, (2 * bb + 1) & 3);
+                    const uint32_t xB0 = u4_at(bb < 2 ? sB0 : sB1, (2 * bb) & 3), xB1 = u4_at(bb < 2 ? sB0 : sB1, (2 * bb + 1) & 3);
                     const uint4 q0 = qa(2 * b, lane), q1 = qa(2 * b + 1, lane);
-                    mma_z(a0, q0, e2m1x2_to_h2(wA), e2m1x2_to_h2(wA >> 8));
-                    mma_z(c0, q0, e2m1x2_to_h2(wB), e2m1x2_to_h2(wB >> 8));
-                    mma_z(a1, q1, e2m1x2_to_h2(wA >> 16), e2m1x2_to_h2(wA >> 24));
-                    mma_z(c1, q1, e2m1x2_to_h2(wB >> 16), e2m1x2_to_h2(wB >> 24));
-                    const float4 dA = *reinterpret_cast<const float4 *>(fA + t * C::KSTRIDE + 4 * b);
-                    const float4 dB = *reinterpret_cast<const float4 *>(fB + t * C::KSTRIDE + 4 * b);
-                    s[0] = fmaf(a1[0] + a1[2], dA.z, fmaf(a0[0] + a0[2], dA.x, s[0]));
-                    s[1] = fmaf(a1[1] + a1[3], dA.w, fmaf(a0[1] + a0[3], dA.y, s[1]));
-                    s[2] = fmaf(c1[0] + c1[2], dB.z, fmaf(c0[0] + c0[2], dB.x, s[2]));
-                    s[3] = fmaf(c1[1] + c1[3], dB.w, fmaf(c0[1] + c0[3], dB.y, s[3]));
+                    float(&ra)[4] = a[b & 1];
+                    float(&rc)[4] = c[b & 1];
+                    const uint32_t kA0 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wA)), u32_as_h2(xA0)));
+                    const uint32_t kA1 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wA >> 8)), u32_as_h2(xA0)));
+                    const uint32_t kA2 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wA >> 16)), u32_as_h2(xA1)));
+                    const uint32_t kA3 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wA >> 24)), u32_as_h2(xA1)));
+                    const uint32_t kB0 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wB)), u32_as_h2(xB0)));
+                    const uint32_t kB1 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wB >> 8)), u32_as_h2(xB0)));
+                    const uint32_t kB2 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wB >> 16)), u32_as_h2(xB1)));
+                    const uint32_t kB3 = h2_as_u32(__hmul2(u32_as_h2(e2m1x2_to_h2(wB >> 24)), u32_as_h2(xB1)));
+                    if (b < 2) {
+                        mma_z(ra, q0, kA0, kA1);
+                        mma_z(rc, q0, kB0, kB1);
+                    } else {
+                        mma_acc(ra, q0, kA0, kA1);
+                        mma_acc(rc, q0, kB0, kB1);
+                    }
+                    mma_acc(ra, q1, kA2, kA3);
+                    mma_acc(rc, q1, kB2, kB3);
                 }
             }
+            s[0] = (a[0][0] + a[0][2]) + (a[1][0] + a[1][2]);
+            s[1] = (a[0][1] + a[0][3]) + (a[1][1] + a[1][3]);
+            s[2] = (c[0][0] + c[0][2]) + (c[1][0] + c[1][2]);
+            s[3] = (c[0][1] + c[0][3]) + (c[1][1] + c[1][3]);
             return;
         }
         {
@@ -574,12 +602,13 @@ template <int FMT> struct QkWarp {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         mx *= inv_sb;                                          // log2 units
-        vmax = max(vmax, item_v_scale_max<FMT>(tp, lane));
+        if constexpr (L::VP != PART_F4) vmax = max(vmax, item_v_scale_max<FMT>(tp, lane));
         const float m_true = m_run + sg;
         // mx is finite on the first item (every row sees key 0); later a row may
         // see none of an item's keys (mx = -inf): nothing moves then
         const float m_new = mx > m_true ? mx + 1.f : m_true;
-        sg = (float)pv_sigma((int)(vmax >> 10));
+        // (nvfp4 values enter the product already scaled, exactly: no shift needed)
+        if constexpr (L::VP != PART_F4) sg = (float)pv_sigma((int)(vmax >> 10));
         const float alpha = ex2(m_run - (m_new - sg));        // 1 when unchanged; 0 on the first item
         l_run *= alpha;
         m_run = m_new - sg;
@@ -681,22 +710,23 @@ template <int FMT> struct PvWarp {
         d8 = e2m1x2_to_h2(v);
         d24 = e2m1x2_to_h2(v >> 8);
     }
+    // The values enter exactly (E2M1 times its E4M3 scale: at most 6 significant
+    // bits, within fp16's normal range), so B is p itself as an fp16 hi/lo pair.
     __device__ __forceinline__ void pv_f4(int b, uint32_t wA, uint32_t wB, uint32_t eA, uint32_t eB, uint32_t mA,
                                           uint32_t mB, uint32_t phA, uint32_t plA, uint32_t phB, uint32_t plB) {
         uint32_t a0, a8, a16, a24, b0, b8, b16, b24;
         f4_pairs(wA, a0, a8, a16, a24);
         f4_pairs(wB, b0, b8, b16, b24);
-        uint32_t hA, lA, hB, lB;
-        pscale(e4m3x2_to_h2(eA) & mA, phA, plA, hA, lA);             // block 2b
-        pscale(e4m3x2_to_h2(eB) & mB, phB, plB, hB, lB);
-        const uint4 m0 = make_uint4(a0, a8, b0, b8);
-        mma_acc(o[2 * b], m0, hA, hB);
-        mma_acc(o[2 * b], m0, lA, lB);
-        pscale(e4m3x2_to_h2(eA >> 16) & mA, phA, plA, hA, lA);       // block 2b + 1
-        pscale(e4m3x2_to_h2(eB >> 16) & mB, phB, plB, hB, lB);
-        const uint4 m1 = make_uint4(a16, a24, b16, b24);
-        mma_acc(o[2 * b + 1], m1, hA, hB);
-        mma_acc(o[2 * b + 1], m1, lA, lB);
+        const __half2 sA = u32_as_h2(e4m3x2_to_h2(eA) & mA), sB = u32_as_h2(e4m3x2_to_h2(eB) & mB);   // block 2b
+        const uint4 m0 = make_uint4(h2_as_u32(__hmul2(u32_as_h2(a0), sA)), h2_as_u32(__hmul2(u32_as_h2(a8), sA)),
+                                    h2_as_u32(__hmul2(u32_as_h2(b0), sB)), h2_as_u32(__hmul2(u32_as_h2(b8), sB)));
+        mma_acc(o[2 * b], m0, phA, phB);
+        mma_acc(o[2 * b], m0, plA, plB);
+        const __half2 tA = u32_as_h2(e4m3x2_to_h2(eA >> 16) & mA), tB = u32_as_h2(e4m3x2_to_h2(eB >> 16) & mB);
+        const uint4 m1 = make_uint4(h2_as_u32(__hmul2(u32_as_h2(a16), tA)), h2_as_u32(__hmul2(u32_as_h2(a24), tA)),
+                                    h2_as_u32(__hmul2(u32_as_h2(b16), tB)), h2_as_u32(__hmul2(u32_as_h2(b24), tB)));
+        mma_acc(o[2 * b + 1], m1, phA, phB);
+        mma_acc(o[2 * b + 1], m1, plA, plB);
     }
 
     // Tiles A, B (consecutive) with p of their tokens 2t, 2t+1.
