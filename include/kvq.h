@@ -6,11 +6,14 @@
  *
  *   q_rotate                      rotate the query by the same transform as K
  *   kv_append                     rotate, quantise and scatter the step's new K/V
- *   paged_decode_attn_{int8,q4_0,k8v4}
+ *   paged_decode_attn_{int8,q4_0,k8v4,fp8,nvfp4}
  *                                 split-K attention over the page table
  *   attn_combine                  merge the splits, un-rotate, write bf16 + f32
- *   paged_decode_step_{int8,q4_0,k8v4}
+ *   paged_decode_step_{int8,q4_0,k8v4,fp8,nvfp4}
  *                                 all of the above for one layer in one launch
+ *   paged_prefill_attn            causal attention of a prompt chunk over the cache
+ *   kvq_resident_*                KV kept in pinned host memory behind a device
+ *                                 page cache (residency table, CLOCK eviction)
  *
  * Sources (web pages, cited by title and section):
  *  [Strata] "KV 沉进内存、显存减半：Strata 让 12 GB 显卡跑满 262K 上下文"

@@ -11,7 +11,6 @@
 // staging buffer, no copy engine) and writes the cache slots.
 #include <algorithm>
 #include <cstring>
-#include <vector>
 
 #include "kvq_internal.cuh"
 
@@ -121,24 +120,40 @@ int kvq_resident_map(void *state, int layer, const int32_t *host_page_table, int
     ResSlot *s = slots_of(h);
     int32_t *t = table_of(h);
 
-    // Validate everything and size the call before touching the state: the
+    // Validate everything and size the call before changing the state: the
     // distinct pages it needs must fit in the cache at once, and the caller's
     // list must hold every page that is not resident.
-    std::vector<int32_t> keys;
     for (int b = 0; b < n_seq; ++b) {
         const int T = seq_len[b];
         if (T < 0 || (int64_t)T > (int64_t)max_pages * PAGE) return KVQ_EINVAL;
         for (int p = 0; p < (T + PAGE - 1) / PAGE; ++p) {
             const int hp = host_page_table[(int64_t)b * max_pages + p];
             if (hp < 0 || hp >= h->n_host_pages) return KVQ_EINVAL;
-            keys.push_back(layer * h->n_host_pages + hp);
         }
     }
-    std::sort(keys.begin(), keys.end());
-    keys.erase(std::unique(keys.begin(), keys.end()), keys.end());
-    if ((int64_t)keys.size() > h->n_slots) return KVQ_ESIZE;
-    int64_t need = 0;
-    for (int32_t k : keys) need += t[k] < 0;
+    // Count distinct pages with temporary marks in the table itself (no
+    // allocation): a missing page -1 becomes -2, a resident page in slot v
+    // becomes -(v + 3); the second pass puts every entry back.
+    int64_t need = 0, resident = 0;
+    for (int pass = 0; pass < 2; ++pass)
+        for (int b = 0; b < n_seq; ++b)
+            for (int p = 0; p < (seq_len[b] + PAGE - 1) / PAGE; ++p) {
+                int32_t &e = t[layer * h->n_host_pages + host_page_table[(int64_t)b * max_pages + p]];
+                if (pass == 0) {
+                    if (e == -1) {
+                        e = -2;
+                        ++need;
+                    } else if (e >= 0) {
+                        e = -(e + 3);
+                        ++resident;
+                    }
+                } else if (e == -2) {
+                    e = -1;
+                } else if (e <= -3) {
+                    e = -(e + 3);
+                }
+            }
+    if (need + resident > h->n_slots) return KVQ_ESIZE;
     if (need > loads_capacity) {
         *n_loads = (int)need;
         return KVQ_ESIZE;
@@ -147,10 +162,13 @@ int kvq_resident_map(void *state, int layer, const int32_t *host_page_table, int
     // Pin the resident part of the batch first, so that no miss of this call
     // evicts a page the same call reads.
     const int epoch = ++h->epoch;
-    for (int32_t k : keys)
-        if (t[k] >= 0) {
-            s[t[k]].ref = 1;
-            s[t[k]].pinned = epoch;
+    for (int b = 0; b < n_seq; ++b)
+        for (int p = 0; p < (seq_len[b] + PAGE - 1) / PAGE; ++p) {
+            const int32_t e = t[layer * h->n_host_pages + host_page_table[(int64_t)b * max_pages + p]];
+            if (e >= 0) {
+                s[e].ref = 1;
+                s[e].pinned = epoch;
+            }
         }
     int nl = 0;
     for (int b = 0; b < n_seq; ++b) {
