@@ -118,11 +118,17 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.t.join(timeout=2)
+        return self.summarize(self.lines, self.uuid)
+
+    @staticmethod
+    def summarize(lines, uuid: str):
+        """Median SM clock, the max clock, and the throttle reasons seen active,
+        over the sample lines of this GPU (uuid; empty = every line)."""
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9 or (self.uuid and self.uuid not in parts[0]):
+            if len(parts) < 9 or (uuid and uuid not in parts[0]):
                 continue
             try:
                 sm.append(float(parts[1]))
