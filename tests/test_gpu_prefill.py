@@ -131,6 +131,16 @@ def test_prefill_key_split_matches_oracle(fmt, n_split):
     _check_rows(w, dw, pos0, out_f, out_bf, list(range(37)), list(range(w.n_kv_heads)))
 
 
+@pytest.mark.parametrize("fmt", ["q4_0", "nvfp4"])
+def test_prefill_from_the_first_token(fmt):
+    """A whole prompt as one chunk (pos0 = 0): row i sees keys 0 .. i only, the
+    first row a single key."""
+    w = _workload(fmt, 12, 2, 300, f"prefill_first_{fmt}")
+    dw, pos0, out_f, out_bf = _prefill(w, 300)
+    assert pos0 == 0
+    _check_rows(w, dw, pos0, out_f, out_bf, [0, 1, 2, 63, 64, 65, 255, 256, 299], list(range(w.n_kv_heads)))
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (8, 1), (6, 2), (14, 2)])
 def test_prefill_group_sizes(Hq, Hkv):
     """Group sizes 1, 8, 3 and 7: the rows r = i G + h of a CTA span token
